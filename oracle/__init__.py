@@ -1,0 +1,201 @@
+"""fp64 CPU oracle for sliding-window attention.
+
+TEST INFRASTRUCTURE: only tests/, the smoke check and the benchmark's
+CPU-baseline leg use this package.  It shares no code with the CUDA path
+(decode_swa_prefill_b200); neither imports the other.
+
+The arithmetic lives in oracle.c (plain C, fp64, two-pass softmax); this module
+only marshals numpy/torch arrays into fp64 C buffers and back.  Each wrapper
+names the page passage its C function follows.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+CAUSAL = 0
+SYMMETRIC = 1
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        c_long, c_int, c_double = ctypes.c_long, ctypes.c_int, ctypes.c_double
+        p = ctypes.c_void_p
+        lib.oracle_in_window.argtypes = [c_long, c_long, c_long, c_long, c_int]
+        lib.oracle_in_window.restype = c_int
+        lib.oracle_allowed.argtypes = [c_long, c_long, c_long, c_long, c_int, p, c_long]
+        lib.oracle_allowed.restype = c_int
+        lib.oracle_mask.argtypes = [p, c_long, c_long, c_int, p, c_long]
+        lib.oracle_mask.restype = None
+        lib.oracle_count_pairs.argtypes = [c_long, c_long, c_int, p, c_long]
+        lib.oracle_count_pairs.restype = ctypes.c_longlong
+        lib.oracle_reach.argtypes = [p, c_long, c_long, c_int]
+        lib.oracle_reach.restype = c_int
+        lib.oracle_slot.argtypes = [c_long, c_long]
+        lib.oracle_slot.restype = c_long
+        lib.oracle_ring_append.argtypes = [p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long]
+        lib.oracle_ring_append.restype = None
+        lib.oracle_swa_prefill.argtypes = [p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
+                                           c_long, c_double, p, c_long, c_int]
+        lib.oracle_swa_prefill.restype = c_int
+        lib.oracle_swa_prefill_global.argtypes = [p, p, p, p, p, p, c_long, c_long, c_long, c_long,
+                                                  c_long, c_long, c_long, c_double, p, c_long, c_int]
+        lib.oracle_swa_prefill_global.restype = c_int
+        lib.oracle_swa_decode.argtypes = [p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
+                                          c_double]
+        lib.oracle_swa_decode.restype = c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    """fp64, C-contiguous numpy copy of a numpy array or (CPU) torch tensor."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _i32(x):
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads():
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+# ------------------------------------------------------------------ masks --
+
+def in_window(i, j, T, W, mode=CAUSAL):
+    """Window membership: causal i-W+1<=j<=i, symmetric |i-j|<=W//2
+    (robocikowo.com "Sliding Window Attention", opening definition)."""
+    return bool(_load().oracle_in_window(i, j, T, W, mode))
+
+
+def mask(T, W, mode=CAUSAL, global_idx=None):
+    """Explicit [T,T] uint8 visibility mask, globals included (Longformer
+    global attention: aivaro.ru answer 629, section 4.3)."""
+    g = 0 if global_idx is None else len(global_idx)
+    gi = None if global_idx is None else _i32(global_idx)
+    out = np.zeros((T, T), dtype=np.uint8)
+    _load().oracle_mask(_ptr(out), T, W, mode, _ptr(gi), g)
+    return out
+
+
+def count_pairs(T, W, mode=CAUSAL, global_idx=None):
+    """Scores computed per layer (Ultralytics glossary, depth section)."""
+    g = 0 if global_idx is None else len(global_idx)
+    gi = None if global_idx is None else _i32(global_idx)
+    return int(_load().oracle_count_pairs(T, W, mode, _ptr(gi), g))
+
+
+def reach(T, W, L):
+    """Last-token reach after 1..L stacked causal layers, by boolean mask
+    products (Ultralytics glossary, depth section)."""
+    out = np.zeros(L, dtype=np.int32)
+    rc = _load().oracle_reach(_ptr(out), T, W, L)
+    assert rc == 0
+    return [int(x) for x in out]
+
+
+def slot(pos, W):
+    """Ring slot of a position (Ultralytics glossary, ring-buffer paragraph)."""
+    return int(_load().oracle_slot(pos, W))
+
+
+def ring_append(k_cache, v_cache, k_new, v_new, pos):
+    """Sequential FIFO append into [B,Hkv,W,d] caches; returns (kc, vc, slots)
+    as new fp64 arrays (robocikowo.com rolling-buffer entry)."""
+    kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    B, Hkv, W, d = kc.shape
+    n = kn.shape[1]
+    slots = np.zeros((B, n), dtype=np.int32)
+    _load().oracle_ring_append(_ptr(kc), _ptr(vc), _ptr(kn), _ptr(vn), _ptr(_i32(pos)), _ptr(slots),
+                               B, n, Hkv, d, W)
+    return kc, vc, slots
+
+
+# ---------------------------------------------------------------- prefill --
+
+def _rows_arg(rows, B, Hq, T):
+    if rows is None:
+        return np.arange(B * Hq * T, dtype=np.int64)
+    return np.ascontiguousarray(rows, dtype=np.int64)
+
+
+def row_ids(b, h, i, Hq, T):
+    """Flattened row id used by the row-subset entry points."""
+    return (np.asarray(b, dtype=np.int64) * Hq + np.asarray(h, dtype=np.int64)) * T + np.asarray(i, dtype=np.int64)
+
+
+def _unflatten(o_rows, lse_rows, rows, full, B, T, Hq, d):
+    if not full:
+        return o_rows, lse_rows
+    # rows enumerate (b, h, i) in order; reshape to [B,T,Hq,d] and [B,Hq,T]
+    o = o_rows.reshape(B, Hq, T, d).transpose(0, 2, 1, 3).copy()
+    lse = lse_rows.reshape(B, Hq, T).copy()
+    return o, lse
+
+
+def swa_prefill(q, k, v, W, scale=None, rows=None, nthreads=None):
+    """Causal SWA (robocikowo.com opening definition; aivaro.ru section 3).
+
+    q [B,T,Hq,d], k/v [B,T,Hkv,d].  rows=None returns the full o [B,T,Hq,d]
+    and lse [B,Hq,T]; otherwise rows are flattened (b*Hq+h)*T+i ids and the
+    result is o [nrows,d], lse [nrows]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = _rows_arg(rows, B, Hq, T)
+    o = np.zeros((len(r), d)); lse = np.zeros(len(r))
+    _load().oracle_swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
+                               float(scale), _ptr(r), len(r), nthreads or default_threads())
+    return _unflatten(o, lse, r, rows is None, B, T, Hq, d)
+
+
+def swa_prefill_global(q, k, v, global_idx, W, scale=None, rows=None, nthreads=None):
+    """Symmetric window |i-j|<=W//2 plus global tokens (aivaro.ru sections
+    4.1 and 4.3).  global_idx [B,g] (g may be 0)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    gi = _i32(global_idx).reshape(B, -1) if global_idx is not None else np.zeros((B, 0), np.int32)
+    g = gi.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = _rows_arg(rows, B, Hq, T)
+    o = np.zeros((len(r), d)); lse = np.zeros(len(r))
+    _load().oracle_swa_prefill_global(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(gi), g,
+                                      B, T, Hq, Hkv, d, W, float(scale), _ptr(r), len(r),
+                                      nthreads or default_threads())
+    return _unflatten(o, lse, r, rows is None, B, T, Hq, d)
+
+
+def swa_decode(q, k_cache, v_cache, pos, scale=None):
+    """One decode step over W-slot rings (Ultralytics ring-buffer paragraph).
+    q [B,Hq,d], caches [B,Hkv,W,d], pos [B] = position of the current token,
+    already appended.  Returns o [B,Hq,d], lse [B,Hq]."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Hq, d = q.shape
+    Hkv, W = kc.shape[1], kc.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, Hq, d)); lse = np.zeros((B, Hq))
+    _load().oracle_swa_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(_i32(pos)), _ptr(o), _ptr(lse),
+                              B, Hq, Hkv, d, W, float(scale))
+    return o, lse

@@ -1,0 +1,297 @@
+/*
+ * Sliding-window attention oracle: plain, slow, fp64, CPU only.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  The CUDA path never links,
+ * includes or calls anything from this directory, and this file includes
+ * nothing from the CUDA path.
+ *
+ * Every floating-point input arrives as fp64 (bf16 or fp32 values upcast
+ * exactly by the caller), every sum is an fp64 sum in index order, and the
+ * softmax is the textbook two-pass form: row maximum first, then exponentials
+ * and their sum, then the weighted sum of value rows divided by that sum.
+ *
+ * Sources (page title, section):
+ *  [P2]  "How sliding window attention works in Mistral and Longformer"
+ *        (aivaro.ru answer 629), sections 2 (idea), 3 (Mistral: the window
+ *        counts the token itself), 4.1 (symmetric W/2 left and right),
+ *        4.3 (Longformer global attention), 9 (pet project: build the mask,
+ *        put -inf at forbidden positions, softmax, weighted sum).
+ *  [P3]  "Sliding Window Attention" (robocikowo.com), opening definition
+ *        paragraph (causal window [i-W+1, i], symmetric [i-W/2, i+W/2],
+ *        -inf logits before the softmax), glossary entries for the binary
+ *        mask, the rolling KV buffer (FIFO) and global tokens.
+ *  [P4]  "Sliding Window Attention" (Ultralytics glossary), section on how
+ *        the window grows with depth (boolean mask, mask products for reach)
+ *        and the ring-buffer paragraph (position i goes to slot i mod w).
+ *
+ * Layouts (the pages fix none): q, o [B,T,Hq,d]; k, v [B,T,Hkv,d];
+ * lse [B,Hq,T]; ring caches [B,Hkv,W,d]; decode q/o [B,Hq,d].
+ * Grouped-query heads: query head h reads kv head floor(h*Hkv/Hq).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_CAUSAL 0
+#define ORACLE_SYMMETRIC 1
+
+/* ---------------------------------------------------------------- masks -- */
+
+/* Window membership of key j for query i [P3 opening paragraph; P2 s.3, 4.1].
+ * causal:    i-W+1 <= j <= i   (W keys including the query itself)
+ * symmetric: i-W/2 <= j <= i+W/2 with W/2 rounded down
+ * Positions outside [0,T) are never keys. */
+int oracle_in_window(long i, long j, long T, long W, int mode)
+{
+    if (j < 0 || j >= T || i < 0 || i >= T) return 0;
+    if (mode == ORACLE_CAUSAL) return (j <= i) && (j >= i - W + 1);
+    long h = W / 2;
+    return (j >= i - h) && (j <= i + h);
+}
+
+static int is_global(long x, const int32_t *gidx, long g)
+{
+    for (long c = 0; c < g; c++)
+        if (gidx[c] == x) return 1;
+    return 0;
+}
+
+/* Longformer-style visibility [P2 s.4.3; P3 glossary entry on global
+ * tokens]: a global token sees every token and every token sees it; all other
+ * pairs follow the symmetric window. */
+int oracle_allowed(long i, long j, long T, long W, int mode, const int32_t *gidx, long g)
+{
+    if (j < 0 || j >= T || i < 0 || i >= T) return 0;
+    if (g > 0 && (is_global(i, gidx, g) || is_global(j, gidx, g))) return 1;
+    return oracle_in_window(i, j, T, W, mode);
+}
+
+/* The explicit [T,T] boolean mask (the brute-force form the pages warn
+ * against for large T; here it is only a checker) [P3 binary-mask entry;
+ * P4 depth section]. */
+void oracle_mask(uint8_t *out, long T, long W, int mode, const int32_t *gidx, long g)
+{
+    for (long i = 0; i < T; i++)
+        for (long j = 0; j < T; j++)
+            out[i * T + j] = (uint8_t)oracle_allowed(i, j, T, W, mode, gidx, g);
+}
+
+/* Number of allowed (query, key) pairs = number of scores one layer computes
+ * [P4 depth section: 58 with the window against 136 fully causal, T=16, W=4]. */
+long long oracle_count_pairs(long T, long W, int mode, const int32_t *gidx, long g)
+{
+    long long n = 0;
+    for (long i = 0; i < T; i++)
+        for (long j = 0; j < T; j++) n += oracle_allowed(i, j, T, W, mode, gidx, g);
+    return n;
+}
+
+/* Reach of the last token through L stacked causal window layers [P4 depth
+ * section]: reach_1 = mask, reach_{l+1} = (mask x reach_l) > 0 as boolean
+ * matrices; out[l-1] = number of tokens the last row of reach_l touches. */
+int oracle_reach(int32_t *out, long T, long W, int L)
+{
+    uint8_t *m = malloc((size_t)T * T), *r = malloc((size_t)T * T), *t = malloc((size_t)T * T);
+    if (!m || !r || !t) { free(m); free(r); free(t); return -1; }
+    oracle_mask(m, T, W, ORACLE_CAUSAL, NULL, 0);
+    memcpy(r, m, (size_t)T * T);
+    for (int l = 0; l < L; l++) {
+        long cnt = 0;
+        for (long j = 0; j < T; j++) cnt += r[(T - 1) * T + j];
+        out[l] = (int32_t)cnt;
+        for (long i = 0; i < T; i++)
+            for (long j = 0; j < T; j++) {
+                int any = 0;
+                for (long k = 0; k < T && !any; k++) any = m[i * T + k] && r[k * T + j];
+                t[i * T + j] = (uint8_t)any;
+            }
+        memcpy(r, t, (size_t)T * T);
+    }
+    free(m); free(r); free(t);
+    return 0;
+}
+
+/* ------------------------------------------------------------ ring cache -- */
+
+/* Ring slot of absolute position pos in a W-slot cache [P4 ring-buffer
+ * paragraph: position i is stored in slot i mod w]. */
+long oracle_slot(long pos, long W) { return pos % W; }
+
+/* Append n new tokens per sequence, one after the other, oldest first; each
+ * write replaces whatever the slot held (FIFO overwrite) [P3 rolling-buffer
+ * entry; P4 ring-buffer paragraph].  kn/vn [B,n,Hkv,d]; caches [B,Hkv,W,d];
+ * pos[b] is the absolute position of token 0 of the batch row; slot_out
+ * (nullable) [B,n] receives the slot each token was written to. */
+void oracle_ring_append(double *kc, double *vc, const double *kn, const double *vn,
+                        const int32_t *pos, int32_t *slot_out,
+                        long B, long n, long Hkv, long d, long W)
+{
+    for (long b = 0; b < B; b++)
+        for (long t = 0; t < n; t++) {
+            long s = oracle_slot((long)pos[b] + t, W);
+            if (slot_out) slot_out[b * n + t] = (int32_t)s;
+            for (long h = 0; h < Hkv; h++) {
+                const double *ksrc = kn + ((b * n + t) * Hkv + h) * d;
+                const double *vsrc = vn + ((b * n + t) * Hkv + h) * d;
+                double *kdst = kc + ((b * Hkv + h) * W + s) * d;
+                double *vdst = vc + ((b * Hkv + h) * W + s) * d;
+                for (long e = 0; e < d; e++) { kdst[e] = ksrc[e]; vdst[e] = vsrc[e]; }
+            }
+        }
+}
+
+/* ------------------------------------------------------ one attention row -- */
+
+/* Softmax-weighted sum over an explicit key list [P2 s.9: scores, forbidden
+ * positions at -inf, softmax, weighted sum; P3: the -inf logits drop out of
+ * the softmax, so only listed keys contribute].  krows/vrows point at the
+ * key/value rows in list order.  Writes o[d] and *lse (natural log of the sum
+ * of exp(score)).  An empty list gives o = 0 and lse = -inf. */
+static void attend_row(const double *q, const double *const *krows, const double *const *vrows,
+                       long nkeys, long d, double scale, double *o, double *lse, double *s)
+{
+    for (long e = 0; e < d; e++) o[e] = 0.0;
+    if (nkeys == 0) { *lse = -INFINITY; return; }
+    double m = -INFINITY;
+    for (long c = 0; c < nkeys; c++) {
+        double acc = 0.0;
+        for (long e = 0; e < d; e++) acc += q[e] * krows[c][e];
+        s[c] = scale * acc;
+        if (s[c] > m) m = s[c];
+    }
+    double l = 0.0;
+    for (long c = 0; c < nkeys; c++) {
+        double p = exp(s[c] - m);
+        l += p;
+        for (long e = 0; e < d; e++) o[e] += p * vrows[c][e];
+    }
+    for (long e = 0; e < d; e++) o[e] /= l;
+    *lse = m + log(l);
+}
+
+/* ---------------------------------------------------------------- prefill -- */
+
+typedef struct {
+    const double *q, *k, *v;
+    double *o, *lse;
+    long B, T, Hq, Hkv, d, W;
+    int mode;
+    const int32_t *gidx; /* [B,g] or NULL */
+    long g;
+    double scale;
+    const int64_t *rows; /* flattened (b*Hq + h)*T + i */
+    long nrows;
+    long next;           /* work counter */
+    pthread_mutex_t mu;
+} prefill_job;
+
+static void prefill_one(prefill_job *J, long r, const double **kr, const double **vr, double *s)
+{
+    long flat = (long)J->rows[r];
+    long i = flat % J->T;
+    long bh = flat / J->T;
+    long h = bh % J->Hq, b = bh / J->Hq;
+    long hk = h * J->Hkv / J->Hq; /* grouped-query head mapping */
+    const int32_t *gb = J->gidx ? J->gidx + b * J->g : NULL;
+    long n = 0;
+    for (long j = 0; j < J->T; j++) {
+        if (!oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0)) continue;
+        kr[n] = J->k + ((b * J->T + j) * J->Hkv + hk) * J->d;
+        vr[n] = J->v + ((b * J->T + j) * J->Hkv + hk) * J->d;
+        n++;
+    }
+    const double *qrow = J->q + ((b * J->T + i) * J->Hq + h) * J->d;
+    double lse;
+    attend_row(qrow, kr, vr, n, J->d, J->scale, J->o + r * J->d, &lse, s);
+    if (J->lse) J->lse[r] = lse;
+}
+
+static void *prefill_worker(void *arg)
+{
+    prefill_job *J = (prefill_job *)arg;
+    const double **kr = malloc(sizeof(double *) * (size_t)J->T);
+    const double **vr = malloc(sizeof(double *) * (size_t)J->T);
+    double *s = malloc(sizeof(double) * (size_t)J->T);
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        long r = J->next;
+        J->next += 16;
+        pthread_mutex_unlock(&J->mu);
+        if (r >= J->nrows) break;
+        long e = r + 16 < J->nrows ? r + 16 : J->nrows;
+        for (; r < e; r++) prefill_one(J, r, kr, vr, s);
+    }
+    free(kr); free(vr); free(s);
+    return NULL;
+}
+
+static int run_prefill(prefill_job *J, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    J->next = 0;
+    pthread_mutex_init(&J->mu, NULL);
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; t++) pthread_create(&th[t], NULL, prefill_worker, J);
+    for (int t = 0; t < nthreads; t++) pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->mu);
+    return 0;
+}
+
+/* Causal sliding-window prefill [P3 opening paragraph; P2 s.3]: for each
+ * requested row (b, h, i) the keys j with i-W+1 <= j <= i of kv head
+ * floor(h*Hkv/Hq).  o: [nrows, d]; lse (nullable): [nrows]. */
+int oracle_swa_prefill(const double *q, const double *k, const double *v, double *o, double *lse,
+                       long B, long T, long Hq, long Hkv, long d, long W, double scale,
+                       const int64_t *rows, long nrows, int nthreads)
+{
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_CAUSAL, NULL, 0, scale, rows, nrows};
+    return run_prefill(&J, nthreads);
+}
+
+/* Symmetric window plus global tokens [P2 s.4.1, 4.3; P3 global-token
+ * entry].  gidx [B,g] lists the global positions of each sequence (g may be
+ * 0: plain symmetric window). */
+int oracle_swa_prefill_global(const double *q, const double *k, const double *v, double *o, double *lse,
+                              const int32_t *gidx, long g,
+                              long B, long T, long Hq, long Hkv, long d, long W, double scale,
+                              const int64_t *rows, long nrows, int nthreads)
+{
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SYMMETRIC, g > 0 ? gidx : NULL, g, scale, rows, nrows};
+    return run_prefill(&J, nthreads);
+}
+
+/* ----------------------------------------------------------------- decode -- */
+
+/* One decode step over the ring cache [P4 ring-buffer paragraph; P5
+ * "Sliding-window and hybrid attention", check-yourself question 1: only the
+ * latest W tokens are kept].  The token at position pos[b] is already in the
+ * cache, so the visible positions are max(0,pos-W+1)..pos, which occupy slots
+ * 0..min(pos+1,W)-1 of the ring.  q/o [B,Hq,d]; caches [B,Hkv,W,d];
+ * lse (nullable) [B,Hq]. */
+int oracle_swa_decode(const double *q, const double *kc, const double *vc, const int32_t *pos,
+                      double *o, double *lse, long B, long Hq, long Hkv, long d, long W, double scale)
+{
+    const double **kr = malloc(sizeof(double *) * (size_t)W);
+    const double **vr = malloc(sizeof(double *) * (size_t)W);
+    double *s = malloc(sizeof(double) * (size_t)W);
+    for (long b = 0; b < B; b++) {
+        long nvalid = (long)pos[b] + 1 < W ? (long)pos[b] + 1 : W;
+        if (pos[b] < 0) nvalid = 0;
+        for (long h = 0; h < Hq; h++) {
+            long hk = h * Hkv / Hq;
+            for (long sl = 0; sl < nvalid; sl++) {
+                kr[sl] = kc + ((b * Hkv + hk) * W + sl) * d;
+                vr[sl] = vc + ((b * Hkv + hk) * W + sl) * d;
+            }
+            double l;
+            attend_row(q + (b * Hq + h) * d, kr, vr, nvalid, d, scale, o + (b * Hq + h) * d, &l, s);
+            if (lse) lse[b * Hq + h] = l;
+        }
+    }
+    free(kr); free(vr); free(s);
+    return 0;
+}
