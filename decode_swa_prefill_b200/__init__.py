@@ -1,0 +1,205 @@
+"""Sliding-window attention on B200: Python binding of libswa.so.
+
+Argument marshalling only.  Every function here takes torch tensors that live
+on a CUDA device, passes their data pointers and sizes to the C ABI declared
+in include/swa.h (same names), and raises SwaError on any non-OK status.  All
+computation happens in the library's CUDA kernels; there is no fallback: if
+libswa.so is missing or cannot be loaded, every call raises.
+
+Layouts: q/o [B,T,Hq,d], k/v [B,T,Hkv,d], lse [B,Hq,T] (fp32), ring caches
+[B,Hkv,W,d], decode q/o [B,Hq,d], positions int32.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SwaError", "load", "library_path", "EXPORTED",
+    "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
+    "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
+    "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libswa.so")
+
+SWA_OK, SWA_ERR_INVALID_ARG, SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA, SWA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
+
+# every symbol include/swa.h declares
+EXPORTED = [
+    "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode_workspace_bytes",
+    "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
+    "swa_set_wait_limit_ns", "swa_status_string",
+]
+
+_lib = None
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, swa_status_string(status), status))
+
+
+def load():
+    """Load libswa.so (built by decode_swa_prefill_b200.build); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError("libswa.so not found at %s; build it with "
+                           "`python -m decode_swa_prefill_b200.build`" % library_path)
+    lib = ctypes.CDLL(library_path)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.swa_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.swa_prefill_global.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.swa_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.swa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
+    lib.swa_mask_export.argtypes = [P, I, I, I, P, I, P]
+    lib.swa_get_device_status.argtypes = [P]
+    lib.swa_debug_expire_wait.argtypes = [I, P]
+    lib.swa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.swa_set_wait_limit_ns.restype = None
+    lib.swa_status_string.argtypes = [I]
+    lib.swa_status_string.restype = ctypes.c_char_p
+    for name in ("swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
+                 "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def swa_status_string(status):
+    return load().swa_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != SWA_OK:
+        raise SwaError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return SWA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return SWA_DTYPE_F32
+    raise SwaError(SWA_ERR_UNSUPPORTED, "dtype %s" % t.dtype)
+
+
+def _need(cond, what):
+    if not cond:
+        raise SwaError(SWA_ERR_INVALID_ARG, what)
+
+
+def _dev_contig(*ts):
+    for t in ts:
+        if t is not None:
+            _need(t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors")
+
+
+def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
+    """Causal sliding-window prefill; returns o (and fills lse when given)."""
+    _dev_contig(q, k, v, o, lse)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, T, Hkv, d) and v.shape == k.shape, "k/v shape")
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
+                            float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_prefill")
+    return o
+
+
+def swa_prefill_global(q, k, v, global_idx, W, scale=None, o=None, lse=None, stream=None):
+    """Symmetric window (half-width W//2) plus global tokens global_idx [B,g] int32."""
+    _dev_contig(q, k, v, o, lse, global_idx)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, T, Hkv, d) and v.shape == k.shape, "k/v shape")
+    g = 0 if global_idx is None else global_idx.shape[-1]
+    if global_idx is not None:
+        _need(global_idx.dtype == torch.int32 and global_idx.shape == (B, g), "global_idx [B,g] int32")
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_global(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                   _ptr(global_idx) if g > 0 else None, g, B, T, Hq, Hkv, d, W,
+                                   float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_prefill_global")
+    return o
+
+
+def swa_cache_append(k_cache, v_cache, k_new, v_new, pos, slot_out=None, stream=None):
+    """Write k_new/v_new [B,n,Hkv,d] into slots (pos[b]+t) mod W of the rings."""
+    _dev_contig(k_cache, v_cache, k_new, v_new, pos, slot_out)
+    B, Hkv, W, d = k_cache.shape
+    n = k_new.shape[1]
+    _need(k_new.shape == (B, n, Hkv, d) and v_new.shape == k_new.shape, "k_new/v_new shape")
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    st = load().swa_cache_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(pos),
+                                 _ptr(slot_out), B, n, Hkv, d, W, _dtype_code(k_cache), _stream(stream))
+    _check(st, "swa_cache_append")
+
+
+def swa_decode_workspace_bytes(B, Hq, Hkv, d, W):
+    return int(load().swa_decode_workspace_bytes(B, Hq, Hkv, d, W))
+
+
+def swa_decode(q, k_cache, v_cache, pos, scale=None, o=None, lse=None, workspace=None, stream=None):
+    """One decode step: q [B,Hq,d] over rings [B,Hkv,W,d]; pos[b] already appended."""
+    _dev_contig(q, k_cache, v_cache, pos, o, lse, workspace)
+    B, Hq, d = q.shape
+    Hkv, W = k_cache.shape[1], k_cache.shape[2]
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    if o is None:
+        o = torch.empty_like(q)
+    need = swa_decode_workspace_bytes(B, Hq, Hkv, d, W)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(pos),
+                           B, Hq, Hkv, d, W, float(scale), _dtype_code(q), _ptr(workspace),
+                           ws_bytes, _stream(stream))
+    _check(st, "swa_decode")
+    return o
+
+
+def swa_mask_export(T, W, symmetric=False, global_idx=None, device=None, stream=None):
+    """[T,T] uint8 visibility mask from the kernels' own predicate (debug)."""
+    device = device or torch.device("cuda")
+    mask = torch.empty((T, T), dtype=torch.uint8, device=device)
+    g = 0 if global_idx is None else global_idx.numel()
+    st = load().swa_mask_export(_ptr(mask), T, W, int(bool(symmetric)),
+                                _ptr(global_idx) if g > 0 else None, g, _stream(stream))
+    _check(st, "swa_mask_export")
+    return mask
+
+
+def swa_get_device_status(stream=None):
+    """Synchronise and read/clear the device status word; returns the status code."""
+    return int(load().swa_get_device_status(_stream(stream)))
+
+
+def swa_debug_expire_wait(timeout_us, stream=None):
+    _check(load().swa_debug_expire_wait(int(timeout_us), _stream(stream)), "swa_debug_expire_wait")
+
+
+def swa_set_wait_limit_ns(ns):
+    load().swa_set_wait_limit_ns(int(ns))

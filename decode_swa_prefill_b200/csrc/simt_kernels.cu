@@ -1,0 +1,478 @@
+// SIMT kernels: mask export, ring-cache append, fp32 prefill, split-K decode
+// over the ring with its LSE merge, and the bounded-wait test hook.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "ptx.cuh"
+#include "swa_internal.h"
+
+namespace swa {
+namespace {
+
+// Is position x one of the g sorted global positions?
+__device__ __forceinline__ bool is_global_pos(const int32_t *gidx, int g, long long x)
+{
+    int lo = 0, hi = g;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (gidx[mid] < x) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo < g && gidx[lo] == x;
+}
+
+// --------------------------------------------------------- mask export --
+// One byte per (i, j), from the band predicate the prefill kernels use plus
+// the global-token rule (robocikowo.com binary-mask and global-token entries).
+__global__ void mask_export_kernel(uint8_t *mask, int T, int left, int right, const int32_t *gidx, int g)
+{
+    const long long n = (long long)T * T;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long i = idx / T, j = idx % T;
+        bool ok = band_contains(i, j, left, right);
+        if (!ok && g > 0) ok = is_global_pos(gidx, g, i) || is_global_pos(gidx, g, j);
+        mask[idx] = ok ? 1 : 0;
+    }
+}
+
+// --------------------------------------------------------- cache append --
+// Token t of row b goes to slot (pos[b]+t) mod W (Ultralytics ring-buffer
+// paragraph); with n > W only the last W tokens are copied, so no two
+// threads write one slot.  16-byte units.
+__global__ void append_kernel(AppendArgs a)
+{
+    const int upr = a.row_bytes / 16;
+    const int n_eff = min(a.n, a.W);
+    const int t0 = a.n - n_eff;
+    const long long total = (long long)a.B * n_eff * a.Hkv * upr;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (a.slot_out) {
+        for (long long idx = tid; idx < (long long)a.B * a.n; idx += stride) {
+            const int b = (int)(idx / a.n), t = (int)(idx % a.n);
+            const long long p = a.pos[b];
+            a.slot_out[idx] = p < 0 ? -1 : (int32_t)((p + t) % a.W);
+        }
+    }
+    for (long long idx = tid; idx < total; idx += stride) {
+        const int u = (int)(idx % upr);
+        long long rest = idx / upr;
+        const int hk = (int)(rest % a.Hkv);
+        rest /= a.Hkv;
+        const int t = t0 + (int)(rest % n_eff);
+        const int b = (int)(rest / n_eff);
+        const long long p = a.pos[b];
+        if (p < 0) {
+            if (u == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+            continue;
+        }
+        const long long slot = (p + t) % a.W;
+        const long long src = (((long long)b * a.n + t) * a.Hkv + hk) * a.row_bytes + u * 16;
+        const long long dst = (((long long)b * a.Hkv + hk) * a.W + slot) * a.row_bytes + u * 16;
+        const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.kn) + src));
+        const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.vn) + src));
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.kc) + dst) = kv;
+        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.vc) + dst) = vv;
+    }
+}
+
+// --------------------------------------------------------- fp32 prefill --
+// One warp per query row, fp32 FMA throughout (no TF32), accurate expf.
+// Keys: the band [i-left, i+right]; for a global row every key; for other
+// rows also the global keys outside the band.
+constexpr int F32_ROWS_PER_CTA = 4;
+
+__global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
+    prefill_f32_kernel(F32PrefillArgs a)
+{
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int i = blockIdx.x * F32_ROWS_PER_CTA + warp;
+    const int h = blockIdx.y, b = blockIdx.z;
+    if (i >= a.T) return;
+    const int hk = h / (a.Hq / a.Hkv);
+    const int32_t *gb = a.gidx ? a.gidx + (long long)b * a.g : nullptr;
+    const bool row_global = gb && is_global_pos(gb, a.g, i);
+    constexpr int EPL = 4; // d <= 128
+    float q[EPL], acc[EPL];
+    const float *qrow = a.q + (((long long)b * a.T + i) * a.Hq + h) * a.d;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const int c = lane + 32 * e;
+        q[e] = c < a.d ? qrow[c] : 0.f;
+        acc[e] = 0.f;
+    }
+    float m = -CUDART_INF_F, l = 0.f;
+    auto visit = [&](long long j) {
+        const float *krow = a.k + (((long long)b * a.T + j) * a.Hkv + hk) * a.d;
+        const float *vrow = a.v + (((long long)b * a.T + j) * a.Hkv + hk) * a.d;
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            const int c = lane + 32 * e;
+            if (c < a.d) dot = fmaf(q[e], krow[c], dot);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float s = dot * a.scale;
+        const float mn = fmaxf(m, s);
+        const float corr = expf(m - mn);
+        const float p = expf(s - mn);
+        l = l * corr + p;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            const int c = lane + 32 * e;
+            acc[e] = acc[e] * corr + (c < a.d ? p * vrow[c] : 0.f);
+        }
+        m = mn;
+    };
+    if (row_global) {
+        for (long long j = 0; j < a.T; ++j) visit(j);
+    } else {
+        const long long lo = max(0LL, (long long)i - a.left);
+        const long long hi = min((long long)a.T - 1, (long long)i + a.right);
+        for (long long j = lo; j <= hi; ++j) visit(j);
+        if (gb)
+            for (int c = 0; c < a.g; ++c)
+                if (!band_contains(i, gb[c], a.left, a.right)) visit(gb[c]);
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float *orow = a.o + (((long long)b * a.T + i) * a.Hq + h) * a.d;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        const int c = lane + 32 * e;
+        if (c < a.d) orow[c] = acc[e] * inv;
+    }
+    if (a.lse && lane == 0) a.lse[((long long)b * a.Hq + h) * a.T + i] = l > 0.f ? m + logf(l) : -CUDART_INF_F;
+}
+
+// ---------------------------------------------------------------- decode --
+// One CTA per (split, kv head, batch row); 4 warps.  Every query head of the
+// GQA group shares the kv head's ring, so one pass over each slot serves all
+// G of them.  Lane l holds elements [l*EPL, (l+1)*EPL) of a head row; a warp
+// reads a whole K or V row per load (coalesced).  A batch of NB = 32/G slots
+// gives NB*G = 32 partial dot products per lane; a reduce-scatter across the
+// warp (31 shuffles) leaves lane L with the full score of (slot L/G, head
+// L%G).  Softmax runs in log2 units with q pre-scaled by scale*log2(e).
+constexpr int DEC_WARPS = 4;
+
+template <typename T>
+struct Ld;
+template <>
+struct Ld<__nv_bfloat16> {
+    template <int EPL>
+    __device__ __forceinline__ static void row(const __nv_bfloat16 *p, float *out)
+    {
+        if constexpr (EPL == 4) {
+            const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+            out[0] = __uint_as_float(u.x << 16);
+            out[1] = __uint_as_float(u.x & 0xffff0000u);
+            out[2] = __uint_as_float(u.y << 16);
+            out[3] = __uint_as_float(u.y & 0xffff0000u);
+        } else if constexpr (EPL == 2) {
+            const uint32_t u = __ldg(reinterpret_cast<const unsigned int *>(p));
+            out[0] = __uint_as_float(u << 16);
+            out[1] = __uint_as_float(u & 0xffff0000u);
+        } else {
+            const unsigned short u = __ldg(reinterpret_cast<const unsigned short *>(p));
+            out[0] = __uint_as_float((uint32_t)u << 16);
+        }
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+template <>
+struct Ld<float> {
+    template <int EPL>
+    __device__ __forceinline__ static void row(const float *p, float *out)
+    {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) out[e] = __ldg(p + e);
+    }
+    __device__ __forceinline__ static void store(float *p, float x) { *p = x; }
+};
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(32 * DEC_WARPS)
+    decode_kernel(DecodeArgs a)
+{
+    constexpr int EPL = D / 32;
+    constexpr int NB = 32 / G;
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int Hq = a.Hq;
+
+    const long long p = a.pos[b];
+    if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+    const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
+    const int chunk = (a.W + a.splits - 1) / a.splits;
+    const int s_begin = split * chunk;
+    const int s_end = min(n_valid, s_begin + chunk);
+
+    const T *qb = static_cast<const T *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
+    const T *kb = static_cast<const T *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+    const T *vb = static_cast<const T *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+
+    float q[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        Ld<T>::template row<EPL>(qb + g * D + lane * EPL, q[g]);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) q[g][e] *= a.scale_log2;
+    }
+    float acc[G][EPL];
+    float m[G], l[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -CUDART_INF_F;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[g][e] = 0.f;
+    }
+
+    for (int base = s_begin + warp * NB; base < s_end; base += DEC_WARPS * NB) {
+        float kr[NB][EPL], vr[NB][EPL];
+#pragma unroll
+        for (int n = 0; n < NB; ++n) {
+            const int sl = min(base + n, s_end - 1); // clamp: masked below
+            Ld<T>::template row<EPL>(kb + (long long)sl * D + lane * EPL, kr[n]);
+            Ld<T>::template row<EPL>(vb + (long long)sl * D + lane * EPL, vr[n]);
+        }
+        // partial dot products, value index n*G + g
+        float v[32];
+#pragma unroll
+        for (int n = 0; n < NB; ++n)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) s = fmaf(q[g][e], kr[n][e], s);
+                v[n * G + g] = s;
+            }
+        // reduce-scatter: after the step with offset k, lane keeps the half
+        // selected by its bit k; finally lane L holds the sum for index L
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1) {
+            const bool upper = (lane & k) != 0;
+#pragma unroll
+            for (int x = 0; x < k; ++x) {
+                const float send = upper ? v[x] : v[x + k];
+                const float keep = upper ? v[x + k] : v[x];
+                v[x] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+            }
+        }
+        const int my_n = lane / G, my_g = lane % G;
+        float sc = (base + my_n < s_end) ? v[0] : -CUDART_INF_F;
+        // per-head batch max over the NB lanes sharing my_g
+        float bm = sc;
+#pragma unroll
+        for (int k = G; k < 32; k <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, k));
+        // running max of my head (m[] is replicated; pick mine)
+        float m_old = m[0];
+#pragma unroll
+        for (int g = 1; g < G; ++g)
+            if (my_g == g) m_old = m[g];
+        const float m_new = fmaxf(m_old, bm);
+        const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+        float pr = ex2_approx(sc - m_use);
+        const float al = ex2_approx(m_old - m_use);
+        float ps = pr;
+#pragma unroll
+        for (int k = G; k < 32; k <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, k);
+        // every lane gets each head's alpha, new max and batch sum
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float alg = __shfl_sync(0xffffffffu, al, g);
+            const float psg = __shfl_sync(0xffffffffu, ps, g);
+            m[g] = __shfl_sync(0xffffffffu, m_new, g);
+            l[g] = l[g] * alg + psg;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[g][e] *= alg;
+        }
+#pragma unroll
+        for (int n = 0; n < NB; ++n)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float pn = __shfl_sync(0xffffffffu, pr, n * G + g);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[g][e] = fmaf(pn, vr[n][e], acc[g][e]);
+            }
+    }
+
+    // merge the warps' partials in shared memory
+    __shared__ float sm_m[DEC_WARPS][G], sm_l[DEC_WARPS][G];
+    __shared__ float sm_acc[DEC_WARPS][G][D];
+    if (lane == 0)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            sm_m[warp][g] = m[g];
+            sm_l[warp][g] = l[g];
+        }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) sm_acc[warp][g][lane * EPL + e] = acc[g][e];
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, e = idx % D;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, sm_m[w][g]);
+        const float Mu = M == -CUDART_INF_F ? 0.f : M;
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) {
+            const float f = ex2_approx(sm_m[w][g] - Mu);
+            L += sm_l[w][g] * f;
+            O += sm_acc[w][g][e] * f;
+        }
+        const int h = hk * G + g;
+        if (a.splits == 1) {
+            T *o = static_cast<T *>(a.o) + ((long long)b * Hq + h) * D;
+            Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
+            if (a.lse && e == 0)
+                a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+        } else {
+            float *part = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
+            part[e] = O;
+            if (e == 0) {
+                part[D] = M;
+                part[D + 1] = L;
+            }
+        }
+    }
+}
+
+// LSE merge of the split partials: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
+template <typename T, int D>
+__global__ void decode_combine_kernel(DecodeArgs a)
+{
+    const int bh = blockIdx.x;
+    const int e = threadIdx.x;
+    const float *part = a.partial + (long long)bh * a.splits * (D + 2);
+    float M = -CUDART_INF_F;
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, part[s * (D + 2) + D]);
+    const float Mu = M == -CUDART_INF_F ? 0.f : M;
+    float L = 0.f, O = 0.f;
+    for (int s = 0; s < a.splits; ++s) {
+        const float f = ex2_approx(part[s * (D + 2) + D] - Mu);
+        L += part[s * (D + 2) + D + 1] * f;
+        O += part[s * (D + 2) + e] * f;
+    }
+    T *o = static_cast<T *>(a.o) + (long long)bh * D;
+    Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
+    if (a.lse && e == 0) a.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
+{
+    dim3 grid(a.splits, a.Hkv, a.B);
+    decode_kernel<T, D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.splits == 1) return e;
+    decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_g(const DecodeArgs &a, cudaStream_t s)
+{
+    switch (a.Hq / a.Hkv) {
+    case 1: return launch_decode_t<T, D, 1>(a, s);
+    case 2: return launch_decode_t<T, D, 2>(a, s);
+    case 4: return launch_decode_t<T, D, 4>(a, s);
+    case 8: return launch_decode_t<T, D, 8>(a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t s)
+{
+    switch (a.d) {
+    case 32: return launch_decode_g<T, 32>(a, s);
+    case 64: return launch_decode_g<T, 64>(a, s);
+    case 128: return launch_decode_g<T, 128>(a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// ------------------------------------------------------ bounded-wait hook --
+__global__ void expire_wait_kernel(DeviceCtl c)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        WaitCtl ctl{&abort_flag, c.status, c.limit_ns};
+        (void)wait_bounded(&bar, 0, ctl); // nothing arrives: expires
+    }
+}
+
+}  // namespace
+
+int decode_splits(int B, int Hq, int Hkv, int d, int W)
+{
+    (void)Hq;
+    (void)d;
+    // enough CTAs for several waves over 148 SMs; each split keeps at least
+    // one full batch of slots per warp
+    const long long units = (long long)B * Hkv;
+    long long want = (148LL * 16 + units - 1) / units;
+    int s = 1;
+    while (s < want && s * 2 * 32 * DEC_WARPS <= W) s *= 2;
+    return s;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
+{
+    const int s = decode_splits(B, Hq, Hkv, d, W);
+    if (s <= 1) return 0;
+    return (size_t)B * Hq * s * (d + 2) * sizeof(float);
+}
+
+cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s)
+{
+    return dtype_bf16 ? launch_decode_d<__nv_bfloat16>(a, s) : launch_decode_d<float>(a, s);
+}
+
+cudaError_t launch_prefill_f32(const F32PrefillArgs &a, cudaStream_t s)
+{
+    dim3 grid((a.T + F32_ROWS_PER_CTA - 1) / F32_ROWS_PER_CTA, a.Hq, a.B);
+    prefill_f32_kernel<<<grid, 32 * F32_ROWS_PER_CTA, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t s)
+{
+    const long long total = (long long)a.B * min(a.n, a.W) * a.Hkv * (a.row_bytes / 16);
+    long long blocks = (total + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    append_kernel<<<(int)blocks, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mask_export(uint8_t *mask, int T, int left, int right, const int32_t *gidx, int g,
+                               cudaStream_t s)
+{
+    const long long n = (long long)T * T;
+    long long blocks = (n + 255) / 256;
+    if (blocks > 148 * 64) blocks = 148 * 64;
+    if (blocks < 1) blocks = 1;
+    mask_export_kernel<<<(int)blocks, 256, 0, s>>>(mask, T, left, right, gidx, g);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_expire_wait(const DeviceCtl &ctl, cudaStream_t s)
+{
+    expire_wait_kernel<<<1, 32, 0, s>>>(ctl);
+    return cudaGetLastError();
+}
+
+}  // namespace swa

@@ -1,0 +1,233 @@
+// The C ABI declared in include/swa.h: argument checks (host only, before any
+// CUDA call), kernel selection and launch on the caller's stream, and the
+// per-device status word that device-side failures are recorded in.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "swa.h"
+#include "swa_internal.h"
+
+// Written by kernels (atomicMax of SWA_STATUS_*), read and cleared by
+// swa_get_device_status.  One instance per device context.
+__device__ int g_swa_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned long long g_wait_limit_ns = 2000000000ull;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+swa_status status_ptr(int **out)
+{
+    static int *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SWA_ERR_CUDA;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_swa_status) != cudaSuccess) return SWA_ERR_CUDA;
+        addr[dev] = static_cast<int *>(p);
+    }
+    *out = addr[dev];
+    return SWA_OK;
+}
+
+swa_status ctl(swa::DeviceCtl *c)
+{
+    c->limit_ns = g_wait_limit_ns;
+    return status_ptr(&c->status);
+}
+
+swa_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return SWA_OK;
+    if (e == cudaErrorInvalidValue) return SWA_ERR_INVALID_ARG;
+    return SWA_ERR_CUDA;
+}
+
+size_t elt_size(swa_dtype dt) { return dt == SWA_DTYPE_BF16 ? 2 : 4; }
+
+bool valid_dtype(swa_dtype dt) { return dt == SWA_DTYPE_BF16 || dt == SWA_DTYPE_F32; }
+
+// Shared checks of the prefill calls.
+swa_status check_prefill(const void *q, const void *k, const void *v, const void *o, const float *lse, int B, int T,
+                         int Hq, int Hkv, int d, int W, float scale, swa_dtype dt)
+{
+    if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || W < 1 || d < 1) return SWA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
+    if (T > (1 << 28)) return SWA_ERR_UNSUPPORTED;
+    if (B == 0 || T == 0) return SWA_OK;
+    if (!q || !k || !v || !o) return SWA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return SWA_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return SWA_ERR_INVALID_ARG;
+    if (dt == SWA_DTYPE_BF16) {
+        if (d != 32 && d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+    } else {
+        if (d > 128 || d % 4 != 0) return SWA_ERR_UNSUPPORTED;
+    }
+    return SWA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *swa_status_string(swa_status s)
+{
+    switch (s) {
+    case SWA_OK: return "ok";
+    case SWA_ERR_INVALID_ARG: return "invalid argument";
+    case SWA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SWA_ERR_CUDA: return "CUDA error";
+    case SWA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+void swa_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns = ns > 0 ? ns : 1; }
+
+swa_status swa_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int T, int Hq,
+                       int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK || B == 0 || T == 0) return st;
+    const int left = W - 1 < T ? W - 1 : T;  // a window wider than T is T
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == SWA_DTYPE_F32) {
+        swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(o), lse, B, T, Hq, Hkv, d, left, 0,
+                              nullptr, 0, scale};
+        return from_cuda(swa::launch_prefill_f32(a, s));
+    }
+    swa::TcPrefillArgs a{};
+    a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv;
+    a.left = left; a.right = 0;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.lse = lse; a.gidx = nullptr; a.g = 0;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+}
+
+swa_status swa_prefill_global(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int32_t *global_idx, int g, int B, int T, int Hq, int Hkv, int d, int W,
+                              float scale, swa_dtype dt, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK) return st;
+    if (g < 0 || g > T) return SWA_ERR_INVALID_ARG;
+    if (g > 0 && (!global_idx || !aligned(global_idx, 4))) return SWA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return SWA_OK;
+    const int half = W / 2 < T ? W / 2 : T;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == SWA_DTYPE_F32) {
+        swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(o), lse, B, T, Hq, Hkv, d, half,
+                              half, g > 0 ? global_idx : nullptr, g, scale};
+        return from_cuda(swa::launch_prefill_f32(a, s));
+    }
+    swa::TcPrefillArgs a{};
+    a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv;
+    a.left = half; a.right = half;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.lse = lse; a.gidx = g > 0 ? global_idx : nullptr; a.g = g;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+}
+
+swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new, const int32_t *pos,
+                            int32_t *slot_out, int B, int n, int Hkv, int d, int W, swa_dtype dt, void *stream)
+{
+    if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (B < 0 || n < 0 || Hkv < 1 || d < 1 || W < 1) return SWA_ERR_INVALID_ARG;
+    if ((d * elt_size(dt)) % 16 != 0) return SWA_ERR_UNSUPPORTED;
+    if (B == 0 || n == 0) return SWA_OK;
+    if (!k_cache || !v_cache || !k_new || !v_new || !pos) return SWA_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+        !aligned(pos, 4) || (slot_out && !aligned(slot_out, 4)))
+        return SWA_ERR_INVALID_ARG;
+    swa::AppendArgs a{k_cache, v_cache, k_new, v_new, pos, slot_out, B, n, Hkv, W,
+                      static_cast<int>(d * elt_size(dt)), {}};
+    swa_status st = ctl(&a.ctl);
+    if (st != SWA_OK) return st;
+    return from_cuda(swa::launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || W < 1 || Hq % Hkv) return 0;
+    return swa::decode_workspace_bytes(B, Hq, Hkv, d, W);
+}
+
+swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
+                      const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (B < 0 || Hq < 1 || Hkv < 1 || W < 1 || d < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (d != 32 && d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+    if (B == 0) return SWA_OK;
+    if (!q || !k_cache || !v_cache || !o || !pos) return SWA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(pos, 4) ||
+        (lse && !aligned(lse, 4)))
+        return SWA_ERR_INVALID_ARG;
+    const size_t need = swa::decode_workspace_bytes(B, Hq, Hkv, d, W);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return SWA_ERR_INVALID_ARG;
+    swa::DecodeArgs a{};
+    a.q = q; a.kc = k_cache; a.vc = v_cache; a.o = o; a.lse = lse; a.pos = pos;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.W = W;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.splits = swa::decode_splits(B, Hq, Hkv, d, W);
+    a.partial = static_cast<float *>(workspace);
+    swa_status st = ctl(&a.ctl);
+    if (st != SWA_OK) return st;
+    return from_cuda(swa::launch_decode(dt == SWA_DTYPE_BF16, a, static_cast<cudaStream_t>(stream)));
+}
+
+swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric, const int32_t *global_idx, int g,
+                           void *stream)
+{
+    if (T < 0 || T > 65536 || W < 1 || (symmetric != 0 && symmetric != 1)) return SWA_ERR_INVALID_ARG;
+    if (g < 0 || g > T || (g > 0 && !symmetric)) return SWA_ERR_INVALID_ARG;
+    if (T == 0) return SWA_OK;
+    if (!mask || (g > 0 && (!global_idx || !aligned(global_idx, 4)))) return SWA_ERR_INVALID_ARG;
+    int left, right;
+    if (symmetric) {
+        left = right = (W / 2 < T ? W / 2 : T);
+    } else {
+        left = W - 1 < T ? W - 1 : T;
+        right = 0;
+    }
+    return from_cuda(
+        swa::launch_mask_export(mask, T, left, right, g > 0 ? global_idx : nullptr, g, static_cast<cudaStream_t>(stream)));
+}
+
+swa_status swa_get_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SWA_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_swa_status, sizeof(int)) != cudaSuccess) return SWA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_swa_status, &zero, sizeof(int)) != cudaSuccess) return SWA_ERR_CUDA;
+    if (v >= SWA_STATUS_TIMEOUT) return SWA_ERR_TIMEOUT;
+    if (v == SWA_STATUS_BAD_INPUT) return SWA_ERR_INVALID_ARG;
+    return SWA_OK;
+}
+
+swa_status swa_debug_expire_wait(int timeout_us, void *stream)
+{
+    if (timeout_us < 1 || timeout_us > 10000000) return SWA_ERR_INVALID_ARG;
+    swa::DeviceCtl c{};
+    swa_status st = status_ptr(&c.status);
+    if (st != SWA_OK) return st;
+    c.limit_ns = static_cast<unsigned long long>(timeout_us) * 1000ull;
+    return from_cuda(swa::launch_debug_expire_wait(c, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

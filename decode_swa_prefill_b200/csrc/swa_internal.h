@@ -1,0 +1,88 @@
+// Internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+// Device status word values (ordered: the worst one wins via atomicMax).
+#define SWA_STATUS_OK 0
+#define SWA_STATUS_BAD_INPUT 1
+#define SWA_STATUS_TIMEOUT 4
+
+namespace swa {
+
+// Key j is visible to query i when i-left <= j <= i+right (both in [0,T)).
+// Causal window W: left = W-1, right = 0.  Symmetric window W: left = right
+// = W/2.  Global tokens are handled by the callers (see the kernels).
+__host__ __device__ __forceinline__ bool band_contains(long long i, long long j, int left, int right)
+{
+    return j >= i - left && j <= i + right;
+}
+
+struct DeviceCtl {
+    int *status;                 // device status word
+    unsigned long long limit_ns; // bounded-wait limit
+};
+
+// ---- tcgen05 prefill (band rows, optional gathered global keys; or dense
+//      global rows) ----
+struct TcPrefillArgs {
+    int B, T, Hq, Hkv;
+    int left, right;          // band of visible keys around each query
+    float scale_log2;         // softmax scale * log2(e)
+    float *lse;               // [B,Hq,T] or null
+    const int32_t *gidx;      // [B,g] global positions or null
+    int g;
+    const void *q, *k, *v;    // raw pointers (gathers)
+    void *o;                  // raw output pointer (scatter in global-row mode)
+    DeviceCtl ctl;
+};
+
+// mode 0: one CTA per (q tile, head, batch) over band tiles (+ one gathered
+//         tile of global keys per 128 globals when gidx != null)
+// mode 1: one CTA per (128 global rows, head, batch): dense rows over all keys
+cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, cudaStream_t s);
+
+// ---- SIMT kernels ----
+struct F32PrefillArgs {
+    const float *q, *k, *v;
+    float *o, *lse;
+    int B, T, Hq, Hkv, d;
+    int left, right;
+    const int32_t *gidx;
+    int g;
+    float scale;
+};
+cudaError_t launch_prefill_f32(const F32PrefillArgs &a, cudaStream_t s);
+
+struct DecodeArgs {
+    const void *q, *kc, *vc;
+    void *o;
+    float *lse;
+    const int32_t *pos;
+    int B, Hq, Hkv, d, W;
+    float scale_log2;
+    float *partial;           // [B,Hq,S,d+2] when S > 1
+    int splits;
+    DeviceCtl ctl;
+};
+int decode_splits(int B, int Hq, int Hkv, int d, int W);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
+cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s);
+
+struct AppendArgs {
+    void *kc, *vc;
+    const void *kn, *vn;
+    const int32_t *pos;
+    int32_t *slot_out;
+    int B, n, Hkv, W;
+    int row_bytes;            // d * element size
+    DeviceCtl ctl;
+};
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t s);
+
+cudaError_t launch_mask_export(uint8_t *mask, int T, int left, int right, const int32_t *gidx, int g,
+                               cudaStream_t s);
+
+cudaError_t launch_debug_expire_wait(const DeviceCtl &ctl, cudaStream_t s);
+
+}  // namespace swa

@@ -1,0 +1,166 @@
+/*
+ * swa.h: sliding-window attention on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The method (as the pages define it):
+ *  - A causal window lets query i see keys i-W+1 .. i: W keys, itself
+ *    included ("Sliding Window Attention", robocikowo.com, opening
+ *    definition; "How sliding window attention works in Mistral and
+ *    Longformer", aivaro.ru, section 3).
+ *  - A symmetric window lets query i see keys i-W/2 .. i+W/2 (W/2 rounded
+ *    down; up to W+1 keys); Longformer adds global tokens that see every
+ *    token and are seen by every token (aivaro.ru, sections 4.1 and 4.3).
+ *  - Scores outside the window are -inf before the softmax, so they take no
+ *    part in it, and the [T,T] score matrix is never formed (robocikowo.com,
+ *    opening definition; aivaro.ru, section 9).
+ *  - Decode keeps a ring of W key/value slots per sequence and head; position
+ *    p lives in slot p mod W, overwriting the oldest entry ("Sliding Window
+ *    Attention", Ultralytics glossary, ring-buffer paragraph).
+ *
+ * Conventions for every call:
+ *  - Every buffer is owned by the caller and lives in device memory unless a
+ *    parameter says otherwise.  The library never allocates device memory.
+ *  - Tensors are dense, row-major, 16-byte aligned, with the layouts given
+ *    below (innermost dimension last).  B batch, T sequence length, Hq query
+ *    heads, Hkv key/value heads (Hq % Hkv == 0; query head h reads kv head
+ *    h / (Hq/Hkv)), d head dimension, W window.
+ *  - bf16 calls run on tcgen05 tensor cores (prefill) or as vectorised SIMT
+ *    (decode); fp32 calls run as SIMT fp32 FMA.  Accumulation is fp32 in
+ *    both, and bf16 outputs are rounded to nearest even.
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
+ *    void*; NULL is the legacy default stream).  Argument errors are detected
+ *    on the host before anything is launched and return SWA_ERR_INVALID_ARG
+ *    or SWA_ERR_UNSUPPORTED; launch failures return SWA_ERR_CUDA.  Errors
+ *    found on the device (a bounded wait that expired, a negative position)
+ *    are recorded in a per-device status word that swa_get_device_status
+ *    reads.  No call aborts the process.
+ */
+#ifndef SWA_H
+#define SWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SWA_OK = 0,
+    SWA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0 ... */
+    SWA_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for (e.g. d) */
+    SWA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    SWA_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired; its outputs are invalid */
+} swa_status;
+
+typedef enum {
+    SWA_DTYPE_F32 = 0,
+    SWA_DTYPE_BF16 = 1
+} swa_dtype;
+
+/*
+ * Causal sliding-window prefill with grouped-query heads.
+ *   o[b,i,h,:] = sum over j in [max(0,i-W+1), i] of
+ *                softmax_j(scale * q[b,i,h,:].k[b,j,hk,:]) * v[b,j,hk,:]
+ * with hk = h / (Hq/Hkv)  (robocikowo.com opening definition; aivaro.ru s.3).
+ *   q, o : [B,T,Hq,d]   k, v : [B,T,Hkv,d]   dtype dt for all four
+ *   lse  : nullable, fp32 [B,Hq,T], natural-log sum of exp(score) per row
+ *   W >= 1 (W >= T is plain causal attention).  scale is normally 1/sqrt(d).
+ *   bf16: d in {32, 64, 128}.  fp32: d <= 128 and d % 4 == 0.
+ */
+swa_status swa_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int T, int Hq, int Hkv, int d, int W, float scale,
+                       swa_dtype dt, void *stream);
+
+/*
+ * Longformer-style bidirectional prefill: symmetric window plus g global
+ * tokens (aivaro.ru sections 4.1 and 4.3; robocikowo.com global-token entry).
+ *   Row i not global: keys j with |i-j| <= W/2, together with every global
+ *   position (a global key inside the band counts once).
+ *   Row i global: every key 0..T-1.
+ *   global_idx : device int32 [B,g], per-sequence positions, strictly
+ *                increasing, each in [0,T); g may be 0 (then global_idx may be
+ *                NULL).  Unsorted or out-of-range entries are undefined.
+ *   Other arguments as swa_prefill; W >= 1 (half-width W/2 rounded down).
+ */
+swa_status swa_prefill_global(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int32_t *global_idx, int g,
+                              int B, int T, int Hq, int Hkv, int d, int W, float scale,
+                              swa_dtype dt, void *stream);
+
+/*
+ * Ring-cache append: token t of batch row b (absolute position pos[b]+t)
+ * goes to slot (pos[b]+t) mod W of that row's ring, overwriting the oldest
+ * entry (Ultralytics ring-buffer paragraph; robocikowo.com rolling-buffer
+ * entry).  When n > W only the last W tokens are written, which leaves the
+ * ring exactly as n one-at-a-time appends would.
+ *   k_cache, v_cache : [B,Hkv,W,d], updated in place
+ *   k_new, v_new     : [B,n,Hkv,d]
+ *   pos              : device int32 [B], >= 0 (a negative entry leaves its row
+ *                      untouched and records SWA_ERR_INVALID_ARG in the
+ *                      device status word)
+ *   slot_out         : nullable device int32 [B,n], receives (pos[b]+t) mod W
+ *   Any d with d * sizeof(dtype) a multiple of 16.
+ */
+swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new,
+                            const int32_t *pos, int32_t *slot_out,
+                            int B, int n, int Hkv, int d, int W, swa_dtype dt, void *stream);
+
+/* Bytes of scratch swa_decode needs for these sizes (0 means none). */
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
+
+/*
+ * One decode step per sequence over the ring (Ultralytics ring-buffer
+ * paragraph; "Sliding-window and hybrid attention", dupenodi.dev, check-
+ * yourself question 1).  The current token (position pos[b]) must already be
+ * appended, so the visible keys are the min(pos[b]+1, W) filled slots
+ * 0 .. min(pos[b]+1,W)-1.
+ *   q, o     : [B,Hq,d]          k_cache, v_cache : [B,Hkv,W,d]
+ *   pos      : device int32 [B], >= 0
+ *   lse      : nullable fp32 [B,Hq]
+ *   workspace: device scratch of at least swa_decode_workspace_bytes(...)
+ *              bytes (may be NULL when that is 0); its contents on entry do
+ *              not matter; calls sharing a workspace must not overlap.
+ *   d in {32, 64, 128}; Hq/Hkv in {1, 2, 4, 8}.
+ */
+swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
+                      const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
+                      swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Debug export of the visibility mask, from the same device predicate the
+ * prefill kernels apply (robocikowo.com binary-mask entry).
+ *   mask : device uint8 [T,T], mask[i*T+j] = 1 when query i may see key j
+ *   symmetric = 0: causal window; 1: symmetric window, with global_idx
+ *   (device int32 [g], sorted, may be NULL when g == 0) as global tokens.
+ *   T <= 65536.
+ */
+swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric,
+                           const int32_t *global_idx, int g, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns SWA_ERR_TIMEOUT if a kernel gave up on a bounded wait since
+ * the last call, SWA_ERR_INVALID_ARG if a kernel met a bad device-side input,
+ * SWA_ERR_CUDA if synchronising failed, else SWA_OK.
+ */
+swa_status swa_get_device_status(void *stream);
+
+/*
+ * Test hook for the failure path: launches one thread that waits on a
+ * barrier nothing will ever complete, through the same bounded wait the
+ * kernels use, with a limit of timeout_us microseconds.  The wait expires,
+ * the kernel records SWA_ERR_TIMEOUT and returns; the context stays usable.
+ */
+swa_status swa_debug_expire_wait(int timeout_us, void *stream);
+
+/* Per-wait limit (nanoseconds) the kernels use; default 2e9 (2 s). */
+void swa_set_wait_limit_ns(unsigned long long ns);
+
+/* Static text for a status code. */
+const char *swa_status_string(swa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H */

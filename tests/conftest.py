@@ -31,3 +31,18 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(autouse=True)
+def _short_device_waits(request):
+    """GPU tests run with a 200 ms bound on every device-side wait, so a
+    broken pipeline shows up as SWA_ERR_TIMEOUT quickly instead of stalling."""
+    if request.node.get_closest_marker("gpu") is None:
+        yield
+        return
+    import decode_swa_prefill_b200 as swa
+    swa.swa_set_wait_limit_ns(200_000_000)
+    yield
+    status = swa.swa_get_device_status()
+    swa.swa_set_wait_limit_ns(2_000_000_000)
+    assert status in (swa.SWA_OK,), "device status word set after test: %d" % status

@@ -1,0 +1,130 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol
+include/swa.h declares, and rejects bad arguments on the host before any CUDA
+call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_swa_prefill_b200 as swa
+from decode_swa_prefill_b200 import build as swa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "swa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    swa_build.build()
+    return swa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(swa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_exports_agree(lib):
+    decl = declared_functions()
+    assert decl == sorted(swa.EXPORTED)
+    for name in decl:
+        assert hasattr(lib, name), name
+
+
+def test_exported_symbols_are_c_linkage():
+    # nm -D lists the plain (unmangled) names
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", swa.library_path], capture_output=True,
+                         text=True, check=True).stdout
+    names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in names, name
+
+
+def test_status_strings(lib):
+    assert swa.swa_status_string(0) == "ok"
+    assert swa.swa_status_string(4) == "device wait timed out"
+    assert swa.swa_status_string(99) == "unknown status"
+
+
+NULL = None
+P = ctypes.c_void_p
+FAKE = ctypes.c_void_p(1 << 20)       # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def prefill(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NULL, B=1, T=16, Hq=4, Hkv=2, d=64, W=4,
+            scale=0.125, dt=1):
+    return lib.swa_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt, NULL)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=NULL), 1), (dict(o=NULL), 1), (dict(k=MISALIGNED), 1), (dict(Hq=3, Hkv=2), 1),
+    (dict(W=0), 1), (dict(W=-5), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1),
+    (dict(scale=float("nan")), 1), (dict(d=48), 2), (dict(d=256), 2), (dict(dt=7), 1),
+    (dict(dt=0, d=130), 2), (dict(dt=0, d=6), 2), (dict(B=-1), 1), (dict(Hkv=0), 1),
+])
+def test_prefill_rejects(lib, kw, expect):
+    assert prefill(lib, **kw) == expect
+
+
+def test_prefill_empty_is_ok_without_touching_memory(lib):
+    # B == 0 or T == 0: nothing to do, even with null pointers
+    assert prefill(lib, q=NULL, k=NULL, v=NULL, o=NULL, B=0) == 0
+    assert prefill(lib, q=NULL, k=NULL, v=NULL, o=NULL, T=0) == 0
+
+
+def test_prefill_global_rejects(lib):
+    f = lib.swa_prefill_global
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 3, 1, 16, 2, 2, 64, 8, 0.125, 1, NULL) == 1  # g>0, no idx
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, FAKE, 17, 1, 16, 2, 2, 64, 8, 0.125, 1, NULL) == 1  # g > T
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, FAKE, -1, 1, 16, 2, 2, 64, 8, 0.125, 1, NULL) == 1
+    assert f(NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, 16, 2, 2, 64, 8, 0.125, 1, NULL) == 0
+
+
+def test_append_rejects(lib):
+    f = lib.swa_cache_append
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1      # no pos
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 2, 1, 8, 4, 64, 1, NULL) == 2        # 8-byte rows
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, NULL, 2, 1, 8, 128, 0, 1, NULL) == 1       # W = 0
+    assert f(FAKE, MISALIGNED, FAKE, FAKE, FAKE, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1
+    assert f(NULL, NULL, NULL, NULL, NULL, NULL, 2, 0, 8, 128, 64, 1, NULL) == 0      # n == 0
+
+
+def test_decode_rejects(lib):
+    f = lib.swa_decode
+    need = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
+    assert need > 0
+    args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, vc=FAKE, o=FAKE, lse=NULL, pos=FAKE, B=64, Hq=32,
+                                  Hkv=8, d=128, W=4096, scale=0.088, dt=1, ws=FAKE, wsb=need), **kw)
+    call = lambda a: f(a["q"], a["kc"], a["vc"], a["o"], a["lse"], a["pos"], a["B"], a["Hq"], a["Hkv"],
+                       a["d"], a["W"], a["scale"], a["dt"], a["ws"], a["wsb"], NULL)
+    assert call(args(ws=NULL)) == 1
+    assert call(args(wsb=need - 1)) == 1
+    assert call(args(Hq=24, Hkv=8)) == 2      # group of 3
+    assert call(args(Hq=36, Hkv=8)) == 1      # not divisible
+    assert call(args(d=96)) == 2
+    assert call(args(pos=NULL)) == 1
+    assert call(args(B=0, q=NULL, kc=NULL, vc=NULL, o=NULL, pos=NULL)) == 0
+
+
+def test_mask_export_rejects(lib):
+    f = lib.swa_mask_export
+    assert f(FAKE, 70000, 4, 0, NULL, 0, NULL) == 1
+    assert f(FAKE, 16, 4, 0, FAKE, 2, NULL) == 1      # globals need the symmetric mode
+    assert f(FAKE, 16, 4, 2, NULL, 0, NULL) == 1
+    assert f(NULL, 0, 4, 0, NULL, 0, NULL) == 0
+
+
+def test_debug_hook_rejects_bad_limits(lib):
+    assert lib.swa_debug_expire_wait(0, NULL) == 1
+    assert lib.swa_debug_expire_wait(10**8, NULL) == 1
+
+
+def test_workspace_sizes(lib):
+    # no workspace when one split suffices; otherwise sized for [B,Hq,S,d+2] fp32
+    big = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
+    assert big % (64 * 32 * 130 * 4) == 0
+    assert lib.swa_decode_workspace_bytes(0, 32, 8, 128, 4096) == 0
