@@ -1,0 +1,480 @@
+"""Benchmark of the sliding-window attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic inputs:
+  1. causal prefill, Mistral-7B shapes (B=1, T=32768, 32/8 heads, d=128, W=4096)
+  2. Longformer-style prefill (B=8, T=4096, 12 heads, d=64, symmetric W=512,
+     16 global tokens)
+  3. ring append of one new token per sequence and
+  4. one decode step over the W=4096-slot ring (64 sequences, 32/8 heads,
+     d=128)
+`value` is the whole step's in-window attention throughput: 4*d FLOPs per
+visible (query, key) pair, summed over the four calls, divided by the step's
+device time.  The components are also timed one by one (CUDA events on the
+launching stream) and reported against their own rooflines: prefill against
+the dense bf16 tensor peak, decode against HBM bandwidth (bytes = the K/V rows
+actually read).  Every input is larger than L2, so no flush is needed between
+steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun): each rank runs its own replica (weak scaling, no
+collective on the data path); ranks are timed on the device and the slowest
+rank's time is reported.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decode_swa_prefill_b200 import workloads as wl  # noqa: E402
+
+METRIC = ("prefill in-window TFLOP/s + % BF16 peak; decode HBM GB/s + % of peak (1 B200)")
+WORKLOAD = "mistral7b_prefill + longformer_prefill_global + ring_append + mistral7b_decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ accounting --
+
+def causal_pairs(T, W):
+    return W * T - W * (W - 1) // 2 if T >= W else T * (T + 1) // 2
+
+
+def global_pairs(T, W, gidx_row):
+    """Visible pairs of one (batch row, head) with a symmetric window and
+    global tokens: band rows see band U G, global rows see all T keys."""
+    h = W // 2
+    i = np.arange(T)
+    band = np.minimum(T - 1, i + h) - np.maximum(0, i - h) + 1
+    g = np.asarray(gidx_row, dtype=np.int64)
+    is_g = np.zeros(T, dtype=bool)
+    is_g[g] = True
+    # globals outside row i's band
+    in_band = (np.abs(i[:, None] - g[None, :]) <= h).sum(axis=1)
+    rows = np.where(is_g, T, band + len(g) - in_band)
+    return int(rows.sum())
+
+
+def step_accounting(inp_lf):
+    P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
+    f_prefill = causal_pairs(P.T, P.W) * P.B * P.Hq * 4 * P.d
+    lf_pairs = sum(global_pairs(L.T, L.W, inp_lf["global_idx"][b].numpy()) for b in range(L.B)) * L.Hq
+    f_lf = lf_pairs * 4 * L.d
+    # decode positions are >= W: every slot is visible
+    f_dec = D.B * D.Hq * D.W * 4 * D.d
+    bytes_dec = D.B * D.Hkv * D.W * D.d * 2 * 2
+    bytes_prefill = (P.B * P.T * (2 * P.Hq + 2 * P.Hkv) * P.d) * 2
+    bytes_lf = (L.B * L.T * (2 * L.Hq + 2 * L.Hkv) * L.d) * 2
+    bytes_append = D.B * D.Hkv * D.d * 2 * 2 * 2
+    return dict(f_prefill=f_prefill, f_lf=f_lf, f_dec=f_dec, bytes_dec=bytes_dec,
+                bytes_prefill=bytes_prefill, bytes_lf=bytes_lf, bytes_append=bytes_append,
+                lf_pairs=lf_pairs)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("prefill_tc.cu", "simt_kernels.cu", "ptx.cuh", "swa_internal.h"):
+        with open(os.path.join(ROOT, "decode_swa_prefill_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary, only if it was taken
+    on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def report(self):
+        if not self.nv or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else None
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- GPU arm --
+
+class Step:
+    """Device-resident inputs/outputs of one step and the calls that run it."""
+
+    def __init__(self, swa, dev):
+        self.swa = swa
+        P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
+        self.host = {"prefill": wl.make(P), "lf": wl.make(L), "dec": wl.make(D)}
+        hp, hl, hd = self.host["prefill"], self.host["lf"], self.host["dec"]
+        self.q, self.k, self.v = (hp[n].to(dev) for n in ("q", "k", "v"))
+        self.o = torch.empty_like(self.q)
+        self.lq, self.lk, self.lv = (hl[n].to(dev) for n in ("q", "k", "v"))
+        self.lg = hl["global_idx"].to(dev)
+        self.lo = torch.empty_like(self.lq)
+        self.dq = hd["q"].to(dev)
+        self.kc, self.vc = hd["k_cache"].to(dev), hd["v_cache"].to(dev)
+        self.kn, self.vn = hd["k_new"].to(dev), hd["v_new"].to(dev)
+        self.pos = hd["pos"].to(dev)
+        self.do = torch.empty_like(self.dq)
+        self.ws = torch.empty(max(1, swa.swa_decode_workspace_bytes(D.B, D.Hq, D.Hkv, D.d, D.W)),
+                              dtype=torch.uint8, device=dev)
+        self.launches_per_step = 1 + 1 + 1 + (2 if self.ws.numel() > 1 else 1)
+
+    def run(self, ev=None):
+        """One step; ev: optional list of 8 events bracketing the 4 calls."""
+        swa, P, L = self.swa, wl.MISTRAL_PREFILL, wl.LONGFORMER
+        if ev: ev[0].record()
+        swa.swa_prefill(self.q, self.k, self.v, P.W, o=self.o)
+        if ev: ev[1].record(); ev[2].record()
+        swa.swa_prefill_global(self.lq, self.lk, self.lv, self.lg, L.W, o=self.lo)
+        if ev: ev[3].record(); ev[4].record()
+        swa.swa_cache_append(self.kc, self.vc, self.kn, self.vn, self.pos)
+        if ev: ev[5].record(); ev[6].record()
+        swa.swa_decode(self.dq, self.kc, self.vc, self.pos, o=self.do, workspace=self.ws)
+        if ev: ev[7].record()
+
+
+def gpu_arm(args, world, rank, local):
+    import decode_swa_prefill_b200 as swa
+    swa.load()
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    st = Step(swa, dev)
+    acc = step_accounting(st.host["lf"])
+    step_flops = acc["f_prefill"] + acc["f_lf"] + acc["f_dec"]
+
+    for _ in range(args.warmup):
+        st.run()
+    torch.cuda.synchronize()
+    assert swa.swa_get_device_status() == 0, "device status after warm-up"
+
+    # ---- device-timed region: exactly K steps ----
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record()
+        for s in range(args.steps):
+            st.run(evs[s])
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    status = swa.swa_get_device_status()
+    assert status == 0, "device status %d after timed region" % status
+    comp = {n: [evs[s][2 * c].elapsed_time(evs[s][2 * c + 1]) for s in range(args.steps)]
+            for c, n in enumerate(("prefill", "longformer", "append", "decode"))}
+    avg = {n: sum(v) / len(v) for n, v in comp.items()}
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = e2e_arm(st, args, world, dev, step_flops)
+
+    peak_t = peaks["bf16_tflops"]
+    peak_h = peaks["hbm_gbs"]
+    pre_tf = acc["f_prefill"] / (avg["prefill"] * 1e-3) / 1e12
+    lf_tf = acc["f_lf"] / (avg["longformer"] * 1e-3) / 1e12
+    dec_gbs = acc["bytes_dec"] / (avg["decode"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs; no weights)",
+        "config": {"workload": WORKLOAD,
+                   "prefill": wl.MISTRAL_PREFILL.name, "longformer": wl.LONGFORMER.name,
+                   "decode": wl.MISTRAL_DECODE.name, "parallelism": "replica per GPU" if world > 1 else "1 GPU",
+                   "l2": "inputs larger than L2 (126 MB) for every kernel; no flush"},
+        "components": {
+            "prefill": {"tflops": round(pre_tf, 2), "ms": round(avg["prefill"], 4),
+                        "frac_of_bf16_peak": round(pre_tf / peak_t, 4), "flops": acc["f_prefill"]},
+            "longformer": {"tflops": round(lf_tf, 2), "ms": round(avg["longformer"], 4),
+                           "frac_of_bf16_peak": round(lf_tf / peak_t, 4),
+                           "gbs": round(acc["bytes_lf"] / (avg["longformer"] * 1e-3) / 1e9, 1),
+                           "flops": acc["f_lf"]},
+            "append": {"us": round(avg["append"] * 1e3, 2)},
+            "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
+                       "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
+                       "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
+        },
+        "roofline": {"kernel": "swa_prefill_tc_kernel<128> (Mistral-7B prefill)", "bound": "tensor",
+                     "achieved": round(pre_tf, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(pre_tf / peak_t, 4), "peak_source": peak_src + " bf16 burst",
+                     "traffic": recorded_traffic("prefill_mistral")},
+        "roofline_decode": {"kernel": "decode_kernel<bf16,128,4> + combine", "bound": "hbm",
+                            "achieved": round(dec_gbs, 1), "peak": peak_h, "unit": "GB/s",
+                            "frac": round(dec_gbs / peak_h, 4), "peak_source": peak_src + " copy",
+                            "traffic": recorded_traffic("decode_mistral")},
+        "clocks": clk.report(),
+        "e2e": e2e,
+        "gpu_launches": st.launches_per_step * args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, world)
+    return line
+
+
+def e2e_arm(st, args, world, dev, step_flops):
+    """Per step: pinned host -> device copies of the step's inputs, the four
+    calls, device -> host copies of the outputs.  The decode ring is resident
+    model state (like weights); the new token's k/v, q and positions are
+    inputs."""
+    hp, hl, hd = st.host["prefill"], st.host["lf"], st.host["dec"]
+    ins = [(hp["q"], st.q), (hp["k"], st.k), (hp["v"], st.v), (hl["q"], st.lq), (hl["k"], st.lk),
+           (hl["v"], st.lv), (hl["global_idx"], st.lg), (hd["q"], st.dq), (hd["k_new"], st.kn),
+           (hd["v_new"], st.vn), (hd["pos"], st.pos)]
+    ins = [(h.pin_memory(), d) for h, d in ins]
+    outs = [(st.o, torch.empty(st.o.shape, dtype=st.o.dtype, pin_memory=True)),
+            (st.lo, torch.empty(st.lo.shape, dtype=st.lo.dtype, pin_memory=True)),
+            (st.do, torch.empty(st.do.shape, dtype=st.do.dtype, pin_memory=True))]
+    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+    d2h = sum(h.numel() * h.element_size() for _, h in outs)
+    steps = max(3, args.steps // 4)
+
+    def one():
+        for h, d in ins:
+            d.copy_(h, non_blocking=True)
+        st.run()
+        for d, h in outs:
+            h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ------------------------------------------------------- oracle (CPU) --
+
+def oracle_sample(budget_s, seed=0):
+    """Run the fp64 oracle on a seeded row sample of every component of the
+    step; returns (in-window FLOPs computed, seconds, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
+    threads = oracle.default_threads()
+    flops, secs = 0, 0.0
+    hp = wl.make(P)
+    hl = wl.make(L)
+    hd = wl.make(D)
+    # rows per component in proportion to their share of a step's FLOPs
+    plan = [("prefill", 0.80), ("longformer", 0.15), ("decode", 0.05)]
+    for name, share in plan:
+        t_budget = budget_s * share
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < t_budget:
+            if name == "prefill":
+                i = rng.integers(P.W, P.T, 64)
+                h = rng.integers(0, P.Hq, 64)
+                oracle.swa_prefill(hp["q"], hp["k"], hp["v"], P.W,
+                                   rows=oracle.row_ids(np.zeros(64, np.int64), h, i, P.Hq, P.T))
+                n += 64 * P.W * 4 * P.d
+            elif name == "longformer":
+                b = rng.integers(0, L.B, 64)
+                h = rng.integers(0, L.Hq, 64)
+                i = rng.integers(0, L.T, 64)
+                oracle.swa_prefill_global(hl["q"], hl["k"], hl["v"], hl["global_idx"], L.W,
+                                          rows=oracle.row_ids(b, h, i, L.Hq, L.T))
+                gi = hl["global_idx"].numpy()
+                for bb, ii in zip(b, i):
+                    row = gi[bb]
+                    if ii in row:
+                        n += L.T * 4 * L.d
+                    else:
+                        hw = L.W // 2
+                        band = min(L.T - 1, ii + hw) - max(0, ii - hw) + 1
+                        n += (band + int((np.abs(row - ii) > hw).sum())) * 4 * L.d
+            else:
+                bsel = rng.integers(0, D.B, 2)
+                oracle.swa_decode(hd["q"][bsel], hd["k_cache"][bsel], hd["v_cache"][bsel],
+                                  hd["pos"][bsel])
+                n += 2 * D.Hq * D.W * 4 * D.d
+        secs += time.perf_counter() - t0
+        flops += n
+    return flops, secs, threads
+
+
+def cpu_baseline(args, world):
+    flops, secs, threads = oracle_sample(args.cpu_seconds)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": "fp64 oracle on seeded row samples of the same step (about %.0f s: "
+                      "Mistral prefill rows past W, Longformer rows, decode sequences), scaled by "
+                      "their in-window FLOPs" % args.cpu_seconds}
+
+
+def reference_arm(args, world, rank):
+    """The oracle as the reference arm: same metric, unit and config, each
+    step a bounded row sample of the step's workload on the host cores."""
+    if rank != 0:
+        return None
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    flops_total, secs_total, threads = 0, 0.0, 1
+    for s in range(args.warmup):
+        oracle_sample(min(per_step, 1.0), seed=1000 + s)
+    for s in range(args.steps):
+        f, t, threads = oracle_sample(per_step, seed=s)
+        flops_total += f
+        secs_total += t
+    v = flops_total / secs_total / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs_total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "prefill": wl.MISTRAL_PREFILL.name,
+                   "longformer": wl.LONGFORMER.name, "decode": wl.MISTRAL_DECODE.name},
+        "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": "each step: fp64 oracle on a seeded row sample (~%.1f s) of the "
+                                   "step's workload" % per_step},
+        "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # rank 0 alone runs the oracle; other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = reference_arm(args, world, rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup()
+    line = gpu_arm(args, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
