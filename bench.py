@@ -448,6 +448,40 @@ def reference_arm(args, world, rank):
     }
 
 
+PROFILE_CASES = {
+    # name: (workload, shape overrides); sizes stay above L2 (126 MB) and a
+    # few GB at most so that an ncu capture of one launch ends quickly
+    "prefill_small": (wl.MISTRAL_PREFILL, {"T": 8192}),
+    "prefill": (wl.MISTRAL_PREFILL, {}),
+    "longformer": (wl.LONGFORMER, {}),
+    "tinymistral": (wl.TINYMISTRAL, {}),
+    "decode": (wl.MISTRAL_DECODE, {}),
+}
+
+
+def profile_case(name, launches):
+    """Run one kernel of the path `launches` times (for ncu captures)."""
+    import dataclasses
+
+    import decode_swa_prefill_b200 as swa
+    w, over = PROFILE_CASES[name]
+    w = dataclasses.replace(w, **over)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = {k: v.to(dev) for k, v in wl.make(w).items()}
+    for _ in range(launches):
+        if w.kind == "prefill":
+            swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W)
+        elif w.kind == "prefill_global":
+            swa.swa_prefill_global(inp["q"], inp["k"], inp["v"], inp["global_idx"], w.W)
+        else:
+            swa.swa_cache_append(inp["k_cache"], inp["v_cache"], inp["k_new"], inp["v_new"], inp["pos"])
+            swa.swa_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["pos"])
+    torch.cuda.synchronize()
+    assert swa.swa_get_device_status() == 0
+    print("profile case %s: %d launches ok" % (name, launches))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,7 +490,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES))
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case, args.launches)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
