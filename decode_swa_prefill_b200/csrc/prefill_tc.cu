@@ -204,10 +204,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         mbar_init(&bars->s_full[0], 1);
         mbar_init(&bars->s_full[1], 1);
-        mbar_init(&bars->p_full, BM);
+        mbar_init(&bars->p_full, BM / 32);
         mbar_init(&bars->pv_done, 1);
         mbar_init(&bars->drain, 1);
-        mbar_init(&bars->epi, BM);
+        mbar_init(&bars->epi, BM / 32);
         bars->abort = 0;
         fence_mbar_init();
     }
@@ -393,9 +393,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
 
             // ---- online softmax (log2 domain, lazy rescale) ----
-            float mx = -CUDART_INF_F;
+            // row max: 8 independent 3-input max chains, then a short tree
+            float mx8[8];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            for (int j = 0; j < 8; ++j) mx8[j] = fmax3(s[j], s[8 + j], s[16 + j]);
+#pragma unroll
+            for (int c = 24; c + 16 <= BN; c += 16)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mx8[j] = fmax3(mx8[j], s[c + j], s[c + 8 + j]);
+#pragma unroll
+            for (int c = 24 + ((BN - 24) / 16) * 16; c < BN; c += 8)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(mx8[j], s[c + j]);
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7]));
             const float mt = mx * a.scale_log2;
             bool rescale_o = false;
             float alpha = 1.f;
@@ -406,13 +417,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 m = mt;
             }
             const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
-            float rs = 0.f;
+            // exponent arguments two at a time (fma.f32x2), four partial sums
+            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+            const float2 nm2 = make_float2(-m_use, -m_use);
+            float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                s[c] = ex2_approx(fmaf(s[c], a.scale_log2, -m_use));
-                rs += s[c];
+            for (int c = 0; c < BN; c += 2) {
+                float2 x = fma2(make_float2(s[c], s[c + 1]), sc2, nm2);
+                s[c] = ex2_approx(x.x);
+                s[c + 1] = ex2_approx(x.y);
+                rs2[(c / 2) & 3] = add2(rs2[(c / 2) & 3], make_float2(s[c], s[c + 1]));
             }
-            l += rs;
+            const float2 r01 = add2(rs2[0], rs2[1]), r23 = add2(rs2[2], rs2[3]);
+            const float2 rsum = add2(r01, r23);
+            l += rsum.x + rsum.y;
 
             // PV of the previous tile must be done: it reads the P buffer and
             // writes O, which a rescale touches
@@ -447,7 +466,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full);
         }
 
         // ---- epilogue ----
@@ -500,7 +520,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const bool direct_store = (w.mode == 1) || (a.gidx != nullptr && a.g > 0);
         if (!direct_store) {
             fence_proxy_async_smem();
-            mbar_arrive(&bars->epi);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->epi);
             if (r == 0 && wait_bounded(&bars->epi, 0, ctl) && !bars->abort) {
                 for (int ch = 0; ch < C::NCH; ++ch)
                     tma_store_4d(&tmO, sQ + ch * C::CH_BYTES, ch * C::E, w.h, w.m0, w.b);
