@@ -201,12 +201,19 @@ def max_over_ranks(x, world):
 
 # ------------------------------------------------------------- GPU arm --
 
+def rank_workload(w, rank):
+    """Each rank of a multi-GPU run processes its own batch: same shapes,
+    seed offset by the rank (weak scaling)."""
+    import dataclasses
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
 class Step:
     """Device-resident inputs/outputs of one step and the calls that run it."""
 
-    def __init__(self, swa, dev):
+    def __init__(self, swa, dev, rank=0):
         self.swa = swa
-        P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
+        P, L, D = (rank_workload(w, rank) for w in (wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE))
         self.host = {"prefill": wl.make(P), "lf": wl.make(L), "dec": wl.make(D)}
         hp, hl, hd = self.host["prefill"], self.host["lf"], self.host["dec"]
         self.q, self.k, self.v = (hp[n].to(dev) for n in ("q", "k", "v"))
@@ -242,7 +249,7 @@ def gpu_arm(args, world, rank, local):
     swa.load()
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
-    st = Step(swa, dev)
+    st = Step(swa, dev, rank)
     acc = step_accounting(st.host["lf"])
     step_flops = acc["f_prefill"] + acc["f_lf"] + acc["f_dec"]
 
