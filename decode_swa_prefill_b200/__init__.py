@@ -18,7 +18,7 @@ __all__ = [
     "SwaError", "load", "library_path", "EXPORTED",
     "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
     "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
-    "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string",
+    "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,7 +31,7 @@ SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 EXPORTED = [
     "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
-    "swa_set_wait_limit_ns", "swa_status_string",
+    "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
 
 _lib = None
@@ -59,6 +59,7 @@ def load():
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.swa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
+    lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P]
     lib.swa_mask_export.argtypes = [P, I, I, I, P, I, P]
     lib.swa_get_device_status.argtypes = [P]
     lib.swa_debug_expire_wait.argtypes = [I, P]
@@ -67,7 +68,7 @@ def load():
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     for name in ("swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
-                 "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
+                 "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -178,6 +179,31 @@ def swa_decode(q, k_cache, v_cache, pos, scale=None, o=None, lse=None, workspace
                            B, Hq, Hkv, d, W, float(scale), _dtype_code(q), _ptr(workspace),
                            ws_bytes, _stream(stream))
     _check(st, "swa_decode")
+    return o
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def swa_decode_noalloc(q, k_cache, v_cache, pos, scale=None, o=None, lse=None, stream=None):
+    """swa_decode without a workspace, for callers that cannot allocate device
+    memory while decoding.  Its scratch is a 16 MiB static device array shared
+    by all calls (overlapping calls on one GPU race); sizes needing more are
+    rejected.  `o` is allocated here only when not given."""
+    _dev_contig(q, k_cache, v_cache, pos, o, lse)
+    B, Hq, d = q.shape
+    Hkv, W = k_cache.shape[1], k_cache.shape[2]
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    need = swa_decode_workspace_bytes(B, Hq, Hkv, d, W)
+    if need > NOALLOC_SCRATCH_BYTES:
+        raise SwaError(SWA_ERR_UNSUPPORTED, "swa_decode_noalloc: these sizes need %d bytes of scratch, "
+                       "above the %d-byte static array" % (need, NOALLOC_SCRATCH_BYTES))
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(pos),
+                                   B, Hq, Hkv, d, W, float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_decode_noalloc")
     return o
 
 

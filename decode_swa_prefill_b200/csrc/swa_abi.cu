@@ -73,6 +73,8 @@ swa_status check_prefill(const void *q, const void *k, const void *v, const void
 
 }  // namespace
 
+int swa::device_ctl(swa::DeviceCtl *c) { return ctl(c) == SWA_OK ? 0 : 1; }
+
 extern "C" {
 
 const char *swa_status_string(swa_status s)

@@ -85,4 +85,8 @@ cudaError_t launch_mask_export(uint8_t *mask, int T, int left, int right, const 
 
 cudaError_t launch_debug_expire_wait(const DeviceCtl &ctl, cudaStream_t s);
 
+// Fills the current device's status-word address and the wait limit; 0 on
+// success.
+int device_ctl(DeviceCtl *c);
+
 }  // namespace swa

@@ -127,6 +127,29 @@ swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, v
                       swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * swa_decode with no workspace argument, for callers that cannot allocate
+ * device memory when they decode: a C host program without an allocator of
+ * its own, a plugin inside a runtime that owns all device memory, or a
+ * serving loop where an allocation could block on the device.  The pages
+ * have no counterpart of this call; it exists only for those callers.
+ *   Arguments, layouts and results as swa_decode.
+ *   Scratch: one static device array of 16 MiB, held by every GPU that loads
+ *   this library until the process exits.  Sizes whose split partials
+ *   (swa_decode_workspace_bytes) exceed 16 MiB are rejected with
+ *   SWA_ERR_UNSUPPORTED before anything runs.  Nothing is allocated.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the array: calls whose kernels overlap on the GPU (two
+ *   streams, or two host threads on one device) race and give wrong results.
+ *   Each call writes every scratch record it reads, so nothing is cleared
+ *   between calls.
+ */
+swa_status swa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
+                              const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
+                              swa_dtype dt, void *stream);
+
+/*
  * Debug export of the visibility mask, from the same device predicate the
  * prefill kernels apply (robocikowo.com binary-mask entry).
  *   mask : device uint8 [T,T], mask[i*T+j] = 1 when query i may see key j
