@@ -3,6 +3,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "swa_internal.h"
 
@@ -342,6 +344,206 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     }
 }
 
+// bf16 decode with 16-byte loads (used when G <= d/8).  A row of d bf16 is
+// read by LPR = d/8 lanes (8 elements, 16 bytes each), so one warp load
+// covers RPW = 32/LPR consecutive ring slots.  Each lane takes NBL = LPR/G
+// slots of a batch (stride RPW), giving NBL*G = LPR partial scores, which a
+// reduce-scatter over the LPR lanes of its row group (log2 LPR shuffles per
+// value pair) turns into one full score per lane.  q.k uses sm_100's mixed
+// precision FMA (bf16 x bf16 + fp32) straight from the packed pairs; P.V
+// runs as paired fp32 FMAs.  Same split-K partials as decode_kernel.
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float c)
+{
+    float d;
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(32 * DEC_WARPS)
+    decode_bf16_kernel(DecodeArgs a)
+{
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPW = 32 / LPR;       // rows per warp load
+    constexpr int NBL = LPR / G;        // slots per lane per batch
+    constexpr int BATCH = NBL * RPW;    // slots per warp per batch
+    static_assert(NBL >= 1 && NBL * G == LPR, "layout");
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int part = lane % LPR;        // which 8 elements of a row
+    const int rgrp = lane / LPR;        // which row of a warp load
+    const int Hq = a.Hq;
+
+    const long long p = a.pos[b];
+    if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+    const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
+    const int chunk = (a.W + a.splits - 1) / a.splits;
+    const int s_begin = split * chunk;
+    const int s_end = min(n_valid, s_begin + chunk);
+
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
+    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+    const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+
+    uint4 q[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) q[g] = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + part * 8));
+    float2 acc[G][4];
+    float m[G], l[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -CUDART_INF_F;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
+    }
+
+    for (int base = s_begin + warp * BATCH; base < s_end; base += DEC_WARPS * BATCH) {
+        uint4 kr[NBL], vr[NBL];
+#pragma unroll
+        for (int n = 0; n < NBL; ++n) {
+            const int sl = min(base + n * RPW + rgrp, s_end - 1); // clamp: masked below
+            kr[n] = __ldg(reinterpret_cast<const uint4 *>(kb + (long long)sl * D + part * 8));
+            vr[n] = __ldg(reinterpret_cast<const uint4 *>(vb + (long long)sl * D + part * 8));
+        }
+        // partial dot products over this lane's 8 elements, index n*G + g
+        float v[LPR];
+#pragma unroll
+        for (int n = 0; n < NBL; ++n)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float t = 0.f;
+                t = dot2_bf16(q[g].x, kr[n].x, t);
+                t = dot2_bf16(q[g].y, kr[n].y, t);
+                t = dot2_bf16(q[g].z, kr[n].z, t);
+                t = dot2_bf16(q[g].w, kr[n].w, t);
+                v[n * G + g] = t;
+            }
+        // reduce-scatter over the LPR lanes of the row group: afterwards
+        // lane part holds the full score of value index part
+#pragma unroll
+        for (int k = LPR / 2; k >= 1; k >>= 1) {
+            const bool upper = (part & k) != 0;
+#pragma unroll
+            for (int x = 0; x < k; ++x) {
+                const float send = upper ? v[x] : v[x + k];
+                const float keep = upper ? v[x + k] : v[x];
+                v[x] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+            }
+        }
+        const int my_n = part / G, my_g = part % G;
+        const float sc = (base + my_n * RPW + rgrp < s_end) ? v[0] * a.scale_log2 : -CUDART_INF_F;
+        // per-head batch max over the lanes holding the same head
+        float bm = sc;
+#pragma unroll
+        for (int k = G; k < 32; k <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, k));
+        float m_old = m[0];
+#pragma unroll
+        for (int g = 1; g < G; ++g)
+            if (my_g == g) m_old = m[g];
+        const float m_new = fmaxf(m_old, bm);
+        const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+        const float pr = ex2_approx(sc - m_use);
+        const float al = ex2_approx(m_old - m_use);
+        float ps = pr;
+#pragma unroll
+        for (int k = G; k < 32; k <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, k);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float alg = __shfl_sync(0xffffffffu, al, g);
+            const float psg = __shfl_sync(0xffffffffu, ps, g);
+            m[g] = __shfl_sync(0xffffffffu, m_new, g);
+            l[g] = l[g] * alg + psg;
+            const float2 a2 = make_float2(alg, alg);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[g][e] = mul2(acc[g][e], a2);
+        }
+        // P.V for this lane's slots (probabilities from its row group)
+#pragma unroll
+        for (int n = 0; n < NBL; ++n) {
+            const float2 v0 = bf16x2_to_float2(vr[n].x), v1 = bf16x2_to_float2(vr[n].y);
+            const float2 v2 = bf16x2_to_float2(vr[n].z), v3 = bf16x2_to_float2(vr[n].w);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float pn = __shfl_sync(0xffffffffu, pr, rgrp * LPR + n * G + g);
+                const float2 p2 = make_float2(pn, pn);
+                acc[g][0] = fma2(p2, v0, acc[g][0]);
+                acc[g][1] = fma2(p2, v1, acc[g][1]);
+                acc[g][2] = fma2(p2, v2, acc[g][2]);
+                acc[g][3] = fma2(p2, v3, acc[g][3]);
+            }
+        }
+    }
+    // sum the row groups' accumulators (same softmax reference per head)
+#pragma unroll
+    for (int k = LPR; k < 32; k <<= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, k);
+                acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, k);
+            }
+
+    // merge the warps' partials in shared memory
+    __shared__ float sm_m[DEC_WARPS][G], sm_l[DEC_WARPS][G];
+    __shared__ float sm_acc[DEC_WARPS][G][D];
+    if (lane == 0)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            sm_m[warp][g] = m[g];
+            sm_l[warp][g] = l[g];
+        }
+    if (rgrp == 0)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sm_acc[warp][g][part * 8 + 2 * e] = acc[g][e].x;
+                sm_acc[warp][g][part * 8 + 2 * e + 1] = acc[g][e].y;
+            }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, e = idx % D;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w2 = 0; w2 < DEC_WARPS; ++w2) M = fmaxf(M, sm_m[w2][g]);
+        const float Mu = M == -CUDART_INF_F ? 0.f : M;
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < DEC_WARPS; ++w2) {
+            const float f = ex2_approx(sm_m[w2][g] - Mu);
+            L += sm_l[w2][g] * f;
+            O += sm_acc[w2][g][e] * f;
+        }
+        const int h = hk * G + g;
+        if (a.splits == 1) {
+            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o) + ((long long)b * Hq + h) * D;
+            o[e] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+            if (a.lse && e == 0)
+                a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+        } else {
+            float *part_out = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
+            part_out[e] = O;
+            if (e == 0) {
+                part_out[D] = M;
+                part_out[D + 1] = L;
+            }
+        }
+    }
+}
+
 // LSE merge of the split partials: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
 template <typename T, int D>
 __global__ void decode_combine_kernel(DecodeArgs a)
@@ -367,7 +569,10 @@ template <typename T, int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
     dim3 grid(a.splits, a.Hkv, a.B);
-    decode_kernel<T, D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8)
+        decode_bf16_kernel<D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    else
+        decode_kernel<T, D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
     decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
