@@ -282,6 +282,7 @@ def gpu_arm(args, world, rank, local):
 
     # ---- end to end through the public API with host buffers ----
     e2e = e2e_arm(st, args, world, dev, step_flops)
+    extra = tinymistral_arm(swa, dev, args)
 
     peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
@@ -303,8 +304,13 @@ def gpu_arm(args, world, rank, local):
             "longformer": {"tflops": round(lf_tf, 2), "ms": round(avg["longformer"], 4),
                            "frac_of_bf16_peak": round(lf_tf / peak_t, 4),
                            "gbs": round(acc["bytes_lf"] / (avg["longformer"] * 1e-3) / 1e9, 1),
+                           # at the ridge: the slower of the two floors over the time taken
+                           "frac_of_min_roofline": round(max(acc["f_lf"] / (peak_t * 1e12),
+                                                             acc["bytes_lf"] / (peak_h * 1e9))
+                                                         / (avg["longformer"] * 1e-3), 4),
                            "flops": acc["f_lf"]},
             "append": {"us": round(avg["append"] * 1e3, 2)},
+            "tinymistral_prefill": extra,
             "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
@@ -324,6 +330,34 @@ def gpu_arm(args, world, rank, local):
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, world)
     return line
+
+
+def tinymistral_arm(swa, dev, args):
+    """TinyMistral-shaped prefill (B=4, T=2048, 32/8 heads, d=32, W=32): HBM
+    bound (25 FLOP per byte), not part of the step.  Its 42 MB fit in L2, so
+    L2 is flushed (256 MB write) before every timed launch."""
+    w = wl.TINYMISTRAL
+    inp = {k: v.to(dev) for k, v in wl.make(w).items()}
+    o = torch.empty_like(inp["q"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, _ = load_peaks()
+    flops = causal_pairs(w.T, w.W) * w.B * w.Hq * 4 * w.d
+    nbytes = w.B * w.T * (2 * w.Hq + 2 * w.Hkv) * w.d * 2
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W, o=o)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
+            "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "bytes": nbytes, "flops": flops,
+            "l2": "flushed before each launch"}
 
 
 def e2e_arm(st, args, world, dev, step_flops):

@@ -3,28 +3,47 @@
 // What it computes (the pages' definition): for query row i, softmax over the
 // keys of its window of scale*q.k, logits outside the window being -inf, then
 // the weighted sum of value rows ("Sliding Window Attention", robocikowo.com,
-// opening definition).  The [T,T] score matrix never exists: each CTA owns
-// one 128-row query tile and streams only the 128-key tiles that intersect
-// the tile's window, skipping every tile that lies fully outside it (the
-// fused-kernel point of the same page and of the Ultralytics glossary's
-// FlashAttention entry).  Work per query tile is O(W*d), total O(T*W*d).
+// opening definition).  The [T,T] score matrix never exists: a CTA streams
+// only the 64-key tiles that intersect its query tiles' windows, skipping
+// every tile that lies fully outside them (the fused-kernel point of the same
+// page and of the Ultralytics glossary's FlashAttention entry).  Work per
+// query tile is O(W*d), total O(T*W*d).
 //
-// CTA anatomy (192 threads):
-//   warps 0-3  softmax + epilogue: thread r owns query row r of the tile,
-//              which is TMEM lane r (warp w may only touch lanes 32w..32w+31)
-//   warp 4     producer: TMA tile loads of Q, K, V (no multicast), or plain
-//              gathers for global keys / global query rows
-//   warp 5     TMEM allocator; lane 0 issues every tcgen05.mma
-// Per key tile t:
-//   S[t&1] = Q K_t^T          (TMEM, fp32, 128 x 128), double buffered so the
-//                             MMA of tile t+1 overlaps the softmax of tile t
-//   softmax: S -> registers (tcgen05.ld), mask (edge tiles only), running
-//            row max in log2 units, P = 2^(S*scale*log2e - m) -> bf16 -> SMEM
-//            (128B-swizzled, K-major, the UMMA A-operand layout)
-//   O += P V_t                (TMEM, fp32, 128 x d)
+// CTA anatomy (352 threads, one CTA per SM), two 128-row query tiles X = A, B
+// that share one kv head, hence every K/V tile: the two query heads of a GQA
+// pair at the same rows, or (odd group size) two consecutive row tiles of one
+// head, whose key ranges are then merged.
+//   warps 0-3  softmax + epilogue of tile A: thread r owns row r = TMEM lane r
+//   warps 4-7  the same for tile B (warp w touches TMEM lanes 32(w%4)...)
+//   warp 8     producer: TMA tile loads of Q, K, V (no multicast), or
+//              cp.async gathers for global keys / global query rows
+//   warp 9     TMEM allocator; with warp 10, the MMA issuers: warp 9 + X runs
+//              tile X's schedule and its lane 0 issues X's tcgen05.mma, so a
+//              wait on one tile never holds up the other tile's MMAs
+// TMEM (all 512 columns):
+//   S[X][b]  columns 128X + 64b: fp32 scores of one 64-key tile, b = buffer
+//   P[X][b]  the first 32 columns of S[X][b]: bf16 probabilities (pairs)
+//   O[X]     columns 256 + 128X: fp32 output accumulator (d <= 128)
+// Per key tile t, for each query tile X, with c = X's running tile count and
+// b = c & 1:
+//   S[X][b] = Q_X K_t^T             (A, B operands from shared memory)
+//   softmax: S -> registers (one TMEM round trip), -inf outside the window
+//            (edge tiles only), running row max in log2 units,
+//            P = 2^(S*scale*log2e - m) -> bf16 -> TMEM over S[X][b]
+//   O[X] += P[X][b] V_t             (A from TMEM, B from shared memory)
+// QK^T of the next tile runs while the softmax of this one works, and the two
+// softmax warpgroups of the CTA hide each other's latencies.  S[X][b] is only
+// recomputed once the PV that read P[X][b] two tiles earlier has completed.
+// Every barrier that alternates between the two S buffers is kept per buffer,
+// so no waiter can fall two phases behind (the parity of an mbarrier phase
+// only names the phase modulo two).
+//
 // The running max is only raised when a tile's max exceeds it by more than
 // 2^8; P then stays <= 256 and O, l share one reference, so the final O/l is
-// exact; raising it rescales l and the O row in TMEM.
+// exact; raising it rescales l and the O row in TMEM.  Per warp, 32-key
+// chunks that no row of the warp can see are skipped.  Half of the
+// exponentials run on the MUFU (ex2.approx), half as a range-reduced cubic on
+// the FMA pipe (exp2_poly2), which roughly halves the MUFU time per tile.
 //
 // Every mbarrier wait is bounded (wait_bounded): on expiry the CTA records
 // SWA_STATUS_TIMEOUT, drains its own in-flight copies and MMAs with a second
@@ -40,58 +59,65 @@ namespace swa {
 namespace {
 
 constexpr int BM = 128;              // query rows per tile (= TMEM lanes)
-constexpr int BN = 128;              // keys per key tile
-constexpr int NSTAGE = 2;            // K/V pipeline depth
-constexpr int NTHREADS = 192;
+constexpr int BN = 64;               // keys per key tile
+constexpr int NSTAGE = 3;            // K and V pipeline depth
+constexpr int NTHREADS = 352;
 constexpr float RESCALE_LOG2 = 8.0f; // raise the running max only beyond 2^8
+constexpr int POLY_EVERY = 4;        // every 4th pair of exponentials on the FMA pipe
+constexpr int SM_SMEM = 228 * 1024;  // shared memory per SM
 
 template <int D>
 struct Cfg {
     static constexpr int RB = (D * 2 >= 128) ? 128 : D * 2; // bytes per swizzled row
     static constexpr int E = RB / 2;                         // elements per chunk row
     static constexpr int NCH = D / E;                        // chunks per head row
-    static constexpr int CH_BYTES = 128 * RB;                // one chunk of a 128-row tile
-    static constexpr int TILE = 128 * D * 2;                 // a 128-row tile of Q, K, V or O
+    static constexpr int QCH = BM * RB;                      // one chunk of a 128-row tile
+    static constexpr int KCH = BN * RB;                      // one chunk of a 64-row tile
+    static constexpr int QTILE = BM * D * 2;
+    static constexpr int KTILE = BN * D * 2;
     static constexpr uint32_t LAYOUT = (RB == 128) ? UMMA_SW128 : UMMA_SW64;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + TILE;
-    static constexpr int OFF_V = OFF_K + NSTAGE * TILE;
-    static constexpr int OFF_P = OFF_V + NSTAGE * TILE;
-    static constexpr int OFF_BAR = OFF_P + BM * BN * 2;
-    // + room to align the base to 1 KiB; at least 120 KiB so that a second CTA
-    // never shares the SM (each CTA takes all 512 TMEM columns)
-    static constexpr int SMEM_NEED = OFF_BAR + 256 + 1024;
+    static constexpr int OFF_Q = 0;                          // Q_A, Q_B
+    static constexpr int OFF_K = OFF_Q + 2 * QTILE;
+    static constexpr int OFF_V = OFF_K + NSTAGE * KTILE;
+    static constexpr int OFF_BAR = OFF_V + NSTAGE * KTILE;
+    // + room to align the base to 1 KiB; more than half the SM's shared
+    // memory so that a second CTA never shares the SM (each CTA takes all
+    // 512 TMEM columns)
+    static constexpr int SMEM_NEED = OFF_BAR + 512 + 1024;
     static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_S = 0;                     // S buffers at columns 0 and 128
-    static constexpr uint32_t COL_O = 256;                   // O accumulator, D columns
     static_assert(D == 32 || D == 64 || D == 128, "head dim");
-    static_assert(SMEM_NEED <= 227 * 1024, "shared memory");
+    static_assert(SMEM_BYTES + 1024 <= SM_SMEM, "fits one SM");
+    static_assert(2 * (SMEM_BYTES + 1024) > SM_SMEM, "never two CTAs per SM");
 };
 
-// Byte offset of element e of row r inside a swizzled [128 rows][D] tile
-// (the layout a TMA SWIZZLE_128B / SWIZZLE_64B load produces).
+__host__ __device__ constexpr uint32_t col_s(int x, int b) { return 128u * x + 64u * b; }
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + 128u * x; }
+
+// Byte offset of element e of row r inside a swizzled [rows][D] tile whose
+// E-element chunks are `ch_bytes` apart (the layout of a TMA SWIZZLE_128B /
+// SWIZZLE_64B load).
 template <int D>
-__device__ __forceinline__ uint32_t tile_offset(int r, int e)
+__device__ __forceinline__ uint32_t tile_offset(int r, int e, int ch_bytes)
 {
     using C = Cfg<D>;
     const int ch = e / C::E;
     const int u = (e % C::E) / 8;
     const int phys = (C::RB == 128) ? (u ^ (r & 7)) : (u ^ ((r >> 1) & 3));
-    return ch * C::CH_BYTES + r * C::RB + phys * 16;
+    return ch * ch_bytes + r * C::RB + phys * 16;
 }
 
 struct Bars {
     uint64_t q_full;
     uint64_t k_full[NSTAGE];
-    uint64_t v_full[NSTAGE];
     uint64_t k_empty[NSTAGE];
+    uint64_t v_full[NSTAGE];
     uint64_t v_empty[NSTAGE];
-    uint64_t s_full[2];
-    uint64_t p_full;
-    uint64_t pv_done;
-    uint64_t drain;
-    uint64_t epi;
+    uint64_t s_full[2][2];   // [tile][buffer]
+    uint64_t p_full[2][2];   // [tile][buffer], one arrival per softmax warp
+    uint64_t pv_done[2][2];  // [tile][buffer]
+    uint64_t drain[2];
+    uint64_t epi[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -105,73 +131,238 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, unsig
     }
 }
 
+// One 128-row query tile of a CTA.
+struct QTile {
+    int h;        // query head
+    int m0;       // first row (band mode)
+    int gt;       // group of 128 global rows (dense-row mode)
+    int nrows;    // real rows
+    int ts, te;   // band key tiles [ts, te) it needs, relative to j_lo
+    bool active;
+};
+
 // The per-CTA work description every role derives identically.
 struct Work {
-    int mode;      // 0 band tile, 1 dense global rows
-    int b, h, hk;
-    int m0;        // first query row (mode 0)
-    int gt;        // global-row group (mode 1)
-    int nrows;     // real rows in the tile (mode 1)
-    int j_lo;      // first key tile
-    int n_band;    // key tiles streamed by TMA
-    int n_glob;    // gathered tiles of global keys (mode 0 with globals)
+    int mode;     // 0 band tiles, 1 dense global rows
+    int b, hk;
+    QTile q[2];
+    int j_lo;     // first band key tile (absolute, 64-key units)
+    int n_band;   // band key tiles streamed by TMA
+    int n_glob;   // gathered tiles of global keys (band mode with globals)
     int n_tiles;
 };
+
+// Does query tile q use key tile t, and which of its tiles is it?
+__device__ __forceinline__ bool tile_active(const QTile &q, int n_band, int t)
+{
+    return q.active && (t >= n_band || (t >= q.ts && t < q.te));
+}
+__device__ __forceinline__ int tile_count(const QTile &q, int n_band, int t)
+{
+    return t < n_band ? t - q.ts : (q.te - q.ts) + (t - n_band);
+}
+__device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
+{
+    return q.active ? (q.te - q.ts) + n_glob : 0;
+}
 
 __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, int n_mode1)
 {
     Work w;
+    const int G = a.Hq / a.Hkv;
+    const bool pair_heads = (G % 2) == 0;
     const int nqt = (a.T + BM - 1) / BM;
     const int nkt = (a.T + BN - 1) / BN;
+    const int ngt = (a.g + BM - 1) / BM;
     int bid = blockIdx.x;
+    for (int x = 0; x < 2; ++x) w.q[x] = QTile{0, 0, 0, 0, 0, 0, false};
     if (bid < n_mode1) {
-        const int ngt = (a.g + BM - 1) / BM;
         w.mode = 1;
-        w.h = bid % a.Hq;
-        w.gt = (bid / a.Hq) % ngt;
-        w.b = bid / (a.Hq * ngt);
-        w.m0 = 0;
-        w.nrows = min(BM, a.g - w.gt * BM);
+        if (pair_heads) {
+            const int hp = bid % (a.Hq / 2);
+            const int gt = (bid / (a.Hq / 2)) % ngt;
+            w.b = bid / ((a.Hq / 2) * ngt);
+            for (int x = 0; x < 2; ++x) w.q[x] = QTile{2 * hp + x, 0, gt, min(BM, a.g - gt * BM), 0, nkt, true};
+        } else {
+            const int h = bid % a.Hq;
+            const int ngp = (ngt + 1) / 2;
+            const int gp = (bid / a.Hq) % ngp;
+            w.b = bid / (a.Hq * ngp);
+            for (int x = 0; x < 2; ++x) {
+                const int gt = 2 * gp + x;
+                if (gt < ngt) w.q[x] = QTile{h, 0, gt, min(BM, a.g - gt * BM), 0, nkt, true};
+            }
+        }
         w.j_lo = 0;
         w.n_band = nkt;
         w.n_glob = 0;
     } else {
         bid -= n_mode1;
         w.mode = 0;
-        w.h = bid % a.Hq;
-        const int qt = (bid / a.Hq) % nqt;
-        w.b = bid / (a.Hq * nqt);
-        w.m0 = qt * BM;
-        w.gt = 0;
-        w.nrows = min(BM, a.T - w.m0);
-        const int lo_key = max(0, w.m0 - a.left);
-        const int hi_key = min(a.T - 1, w.m0 + BM - 1 + a.right);
-        w.j_lo = lo_key / BN;
-        w.n_band = hi_key / BN - w.j_lo + 1;
+        if (pair_heads) {
+            const int hp = bid % (a.Hq / 2);
+            const int qt = (bid / (a.Hq / 2)) % nqt;
+            w.b = bid / ((a.Hq / 2) * nqt);
+            for (int x = 0; x < 2; ++x)
+                w.q[x] = QTile{2 * hp + x, qt * BM, 0, min(BM, a.T - qt * BM), 0, 0, true};
+        } else {
+            const int h = bid % a.Hq;
+            const int nqp = (nqt + 1) / 2;
+            const int qp = (bid / a.Hq) % nqp;
+            w.b = bid / (a.Hq * nqp);
+            for (int x = 0; x < 2; ++x) {
+                const int qt = 2 * qp + x;
+                if (qt < nqt) w.q[x] = QTile{h, qt * BM, 0, min(BM, a.T - qt * BM), 0, 0, true};
+            }
+        }
+        int lo = a.T, hi = -1;
+        int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+        for (int x = 0; x < 2; ++x) {
+            if (!w.q[x].active) continue;
+            lo_x[x] = max(0, w.q[x].m0 - a.left);
+            hi_x[x] = min(a.T - 1, w.q[x].m0 + BM - 1 + a.right);
+            lo = min(lo, lo_x[x]);
+            hi = max(hi, hi_x[x]);
+        }
+        w.j_lo = lo / BN;
+        w.n_band = hi / BN - w.j_lo + 1;
+        for (int x = 0; x < 2; ++x)
+            if (w.q[x].active) {
+                w.q[x].ts = lo_x[x] / BN - w.j_lo;
+                w.q[x].te = hi_x[x] / BN - w.j_lo + 1;
+            }
         w.n_glob = (a.gidx != nullptr && a.g > 0) ? (a.g + BN - 1) / BN : 0;
     }
-    w.hk = w.h / (a.Hq / a.Hkv);
+    w.hk = w.q[0].h / G;
     w.n_tiles = w.n_band + w.n_glob;
     return w;
 }
 
-// Producer-warp gather of up to 128 rows (positions from `rows_idx`) of one
-// head into a swizzled tile; rows past `nrows` are zero.  All 32 lanes.
+// Key columns of tile t that the MMAs compute (a multiple of 32): all 64 of a
+// band tile, the real global keys of a gathered tile rounded up.
+__device__ __forceinline__ int tile_cols(const Work &w, const TcPrefillArgs &a, int t)
+{
+    if (t < w.n_band) return BN;
+    const int n = min(BN, a.g - (t - w.n_band) * BN);
+    return (n + 31) & ~31;
+}
+
+// Producer-warp gather of up to `rows` rows (positions from `rows_idx`) of
+// one head into a swizzled tile with 16-byte cp.async copies, all in flight
+// at once; rows past `nrows` are zero-filled.  All 32 lanes.
 template <int D>
-__device__ __forceinline__ void gather_tile(uint8_t *dst, const __nv_bfloat16 *base, const int32_t *rows_idx,
-                                            int nrows, int b, int T, int H, int head, int lane)
+__device__ __forceinline__ void gather_tile(uint8_t *dst, int rows, int ch_bytes, const __nv_bfloat16 *base,
+                                            const int32_t *rows_idx, int nrows, int b, int T, int H, int head,
+                                            int lane)
 {
     constexpr int GR = D / 8; // 16-byte granules per row
-    for (int idx = lane; idx < 128 * GR; idx += 32) {
+    for (int idx = lane; idx < rows * GR; idx += 32) {
         const int r = idx / GR, u = idx % GR;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (r < nrows) {
-            const long long pos = rows_idx[r];
-            const __nv_bfloat16 *src = base + (((long long)b * T + pos) * H + head) * D + u * 8;
-            val = __ldg(reinterpret_cast<const uint4 *>(src));
-        }
-        *reinterpret_cast<uint4 *>(dst + tile_offset<D>(r, u * 8)) = val;
+        const long long pos = r < nrows ? rows_idx[r] : 0;
+        const __nv_bfloat16 *src = base + (((long long)b * T + pos) * H + head) * D + u * 8;
+        cp_async16(dst + tile_offset<D>(r, u * 8, ch_bytes), src, r < nrows ? 16u : 0u);
     }
+    cp_async_wait_all();
+}
+
+// Everything the softmax of one 64-key tile needs besides the scores.
+struct TileCtx {
+    uint32_t s_addr;      // TMEM address of this warp's lanes of S[X][b]
+    int c_lo, c_hi;       // live 32-key chunks of the warp
+    int col_lo, col_hi;   // visible columns of this row (band / dense tiles)
+    bool by_range;        // mask by [col_lo, col_hi] (else: global-key tile)
+    int gc_base;          // first global index of a gathered tile
+    long long i_row;
+};
+
+// Softmax of one tile for one row: scores -> running max / sum -> P (bf16)
+// over the first 32 columns of the tile's TMEM buffer.  FULL: every key of
+// the tile is visible to every row of the warp (no masking, all chunks live),
+// the common case, compiled without any of the masking branches.
+template <bool FULL>
+__device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillArgs &a, const int32_t *gb, float &m,
+                                             float &l, bool &rescale, float &alpha, bool first)
+{
+    auto live = [&](int cc) { return FULL || (cc >= k.c_lo && cc <= k.c_hi); };
+    float sr[BN];
+#pragma unroll
+    for (int cc = 0; cc < BN / 32; ++cc)
+        if (live(cc)) tmem_ld32(k.s_addr + cc * 32, sr + cc * 32);
+    tmem_ld_wait_dep(sr);
+#pragma unroll
+    for (int cc = 1; cc < BN / 32; ++cc) reg_fence32(sr + cc * 32);
+    if (!FULL) {
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) {
+            if (!live(cc)) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sr[cc * 32 + e] = -CUDART_INF_F;
+            } else if (k.by_range) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int xx = cc * 32 + e;
+                    if (xx < k.col_lo || xx > k.col_hi) sr[xx] = -CUDART_INF_F;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int gc = k.gc_base + cc * 32 + e;
+                    const bool keep = gc < a.g && !band_contains(k.i_row, __ldg(gb + gc), a.left, a.right);
+                    if (!keep) sr[cc * 32 + e] = -CUDART_INF_F;
+                }
+            }
+        }
+    }
+    float mx4[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mx4[j] = fmax3(sr[j], sr[4 + j], sr[8 + j]);
+#pragma unroll
+    for (int cc = 12; cc + 8 <= BN; cc += 8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], sr[cc + j], sr[cc + 4 + j]);
+#pragma unroll
+    for (int cc = 12 + ((BN - 12) / 8) * 8; cc < BN; cc += 4)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx4[j] = fmaxf(mx4[j], sr[cc + j]);
+    const float mt = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * a.scale_log2;
+    rescale = false;
+    alpha = 1.f;
+    if (mt > m + RESCALE_LOG2) {
+        alpha = ex2_approx(m - mt);     // 0 when m was -inf
+        l *= alpha;
+        rescale = !first;
+        m = mt;
+    }
+    const float ref = (m == -CUDART_INF_F) ? 0.f : m;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+    const float2 nr2 = make_float2(-ref, -ref);
+    float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t pk[16];
+        if (live(cc)) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const int xx = cc * 32 + e;
+                float2 y = fma2(make_float2(sr[xx], sr[xx + 1]), sc2, nr2);
+                if ((e / 2) % POLY_EVERY == POLY_EVERY - 1) {
+                    y = exp2_poly2(y);
+                } else {
+                    y.x = ex2_approx(y.x);
+                    y.y = ex2_approx(y.y);
+                }
+                if (e & 2) acc2b = add2(acc2b, y);
+                else acc2 = add2(acc2, y);
+                pk[e / 2] = pack_bf16x2(y.x, y.y);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        }
+        tmem_st16u(k.s_addr + cc * 16, pk);
+    }
+    const float2 tot = add2(acc2, acc2b);
+    l += tot.x + tot.y;
 }
 
 template <int D>
@@ -183,10 +374,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem + C::OFF_Q;
+    uint8_t *sQ = smem + C::OFF_Q;   // Q_X at sQ + X * QTILE
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
-    uint8_t *sP = smem + C::OFF_P;
     Bars *bars = reinterpret_cast<Bars *>(smem + C::OFF_BAR);
 
     const int warp = threadIdx.x / 32;
@@ -198,26 +388,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(&bars->q_full, 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 2);   // one commit per MMA issuer
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->k_empty[s], 1);
-            mbar_init(&bars->v_empty[s], 1);
+            mbar_init(&bars->v_empty[s], 2);
         }
-        mbar_init(&bars->s_full[0], 1);
-        mbar_init(&bars->s_full[1], 1);
-        mbar_init(&bars->p_full, BM / 32);
-        mbar_init(&bars->pv_done, 1);
-        mbar_init(&bars->drain, 1);
-        mbar_init(&bars->epi, BM / 32);
+        for (int x = 0; x < 2; ++x) {
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&bars->s_full[x][b], 1);
+                mbar_init(&bars->p_full[x][b], BM / 32);
+                mbar_init(&bars->pv_done[x][b], 1);
+            }
+            mbar_init(&bars->epi[x], BM / 32);
+            mbar_init(&bars->drain[x], 1);
+        }
         bars->abort = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
         prefetch_tensormap(&tmO);
     }
-    if (warp == 5) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    if (warp == 9) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -225,257 +418,262 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     const int32_t *gb = a.gidx ? a.gidx + (long long)w.b * a.g : nullptr;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------ producer --
-        int issued[NSTAGE] = {0, 0}, vissued[NSTAGE] = {0, 0};
+        int kiss[NSTAGE] = {}, viss[NSTAGE] = {};
         bool ok = true;
         if (w.mode == 0) {
             if (lane == 0) {
-                mbar_expect_tx(&bars->q_full, C::TILE);
-                for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_load_4d(sQ + ch * C::CH_BYTES, &tmQ, &bars->q_full, ch * C::E, w.h, w.m0, w.b);
+                int nq = 0;
+                for (int x = 0; x < 2; ++x) nq += w.q[x].active ? 1 : 0;
+                mbar_expect_tx(&bars->q_full, nq * C::QTILE);
+                for (int x = 0; x < 2; ++x)
+                    if (w.q[x].active)
+                        for (int ch = 0; ch < C::NCH; ++ch)
+                            tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, &tmQ, &bars->q_full, ch * C::E, w.q[x].h,
+                                        w.q[x].m0, w.b);
             }
         } else {
-            gather_tile<D>(sQ, static_cast<const __nv_bfloat16 *>(a.q), gb + w.gt * BM, w.nrows, w.b, a.T, a.Hq,
-                           w.h, lane);
+            for (int x = 0; x < 2; ++x)
+                if (w.q[x].active)
+                    gather_tile<D>(sQ + x * C::QTILE, BM, C::QCH, static_cast<const __nv_bfloat16 *>(a.q),
+                                   gb + w.q[x].gt * BM, w.q[x].nrows, w.b, a.T, a.Hq, w.q[x].h, lane);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->q_full);
         }
         for (int t = 0; t < w.n_tiles && ok; ++t) {
+            const bool band = t < w.n_band;
+            const int key0 = (w.j_lo + t) * BN;
+            const int gt = t - w.n_band;
+            const int nr = band ? 0 : min(BN, a.g - gt * BN);
             const int st = t % NSTAGE;
-            const uint32_t ph = (t / NSTAGE) & 1;
-            ok = warp_wait_bounded(&bars->k_empty[st], ph ^ 1, ctl);
+            const uint32_t par = ((t / NSTAGE) & 1) ^ 1;
+            ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
             if (!ok) break;
-            if (t < w.n_band) {
-                const int key0 = (w.j_lo + t) * BN;
+            if (band) {
                 if (lane == 0) {
-                    mbar_expect_tx(&bars->k_full[st], C::TILE);
+                    mbar_expect_tx(&bars->k_full[st], C::KTILE);
                     for (int ch = 0; ch < C::NCH; ++ch)
-                        tma_load_4d(sK + st * C::TILE + ch * C::CH_BYTES, &tmK, &bars->k_full[st], ch * C::E, w.hk,
-                                    key0, w.b);
-                }
-                issued[st]++;
-                ok = warp_wait_bounded(&bars->v_empty[st], ph ^ 1, ctl);
-                if (!ok) break;
-                if (lane == 0) {
-                    mbar_expect_tx(&bars->v_full[st], C::TILE);
-                    for (int ch = 0; ch < C::NCH; ++ch)
-                        tma_load_4d(sV + st * C::TILE + ch * C::CH_BYTES, &tmV, &bars->v_full[st], ch * C::E, w.hk,
+                        tma_load_4d(sK + st * C::KTILE + ch * C::KCH, &tmK, &bars->k_full[st], ch * C::E, w.hk,
                                     key0, w.b);
                 }
             } else {
-                const int gt = t - w.n_band;
-                const int nr = min(BN, a.g - gt * BN);
-                ok = warp_wait_bounded(&bars->v_empty[st], ph ^ 1, ctl);
-                if (!ok) break;
-                issued[st]++;
-                gather_tile<D>(sK + st * C::TILE, static_cast<const __nv_bfloat16 *>(a.k), gb + gt * BN, nr, w.b,
-                               a.T, a.Hkv, w.hk, lane);
-                gather_tile<D>(sV + st * C::TILE, static_cast<const __nv_bfloat16 *>(a.v), gb + gt * BN, nr, w.b,
-                               a.T, a.Hkv, w.hk, lane);
+                gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
+                               gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bars->k_full[st]);
-                    mbar_arrive(&bars->v_full[st]);
-                }
+                if (lane == 0) mbar_arrive(&bars->k_full[st]);
             }
-            vissued[st]++;
+            kiss[st]++;
+            ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
+            if (!ok) break;
+            if (band) {
+                if (lane == 0) {
+                    mbar_expect_tx(&bars->v_full[st], C::KTILE);
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        tma_load_4d(sV + st * C::KTILE + ch * C::KCH, &tmV, &bars->v_full[st], ch * C::E, w.hk,
+                                    key0, w.b);
+                }
+            } else {
+                gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
+                               gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->v_full[st]);
+            }
+            viss[st]++;
         }
         if (!ok && lane == 0) {
             // let our own copies land before the CTA's shared memory goes away
-            for (int s = 0; s < NSTAGE; ++s)
-            {
-                if (issued[s] > 0) drain_wait(&bars->k_full[s], (issued[s] - 1) & 1, a.ctl.limit_ns);
-                if (vissued[s] > 0) drain_wait(&bars->v_full[s], (vissued[s] - 1) & 1, a.ctl.limit_ns);
+            for (int s = 0; s < NSTAGE; ++s) {
+                if (kiss[s] > 0) drain_wait(&bars->k_full[s], (kiss[s] - 1) & 1, a.ctl.limit_ns);
+                if (viss[s] > 0) drain_wait(&bars->v_full[s], (viss[s] - 1) & 1, a.ctl.limit_ns);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9 || warp == 10) {
         // ----------------------------------------------------------- MMA --
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = umma_idesc_bf16(BM, BN, 0, 0);
-            constexpr uint32_t idesc_pv = umma_idesc_bf16(BM, D, 0, 1);
-            const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
-            const uint32_t p_base = smem_u32(sP);
-            bool ok = wait_bounded(&bars->q_full, 0, ctl);
-            tc_fence_after();
-            auto issue_pv = [&](int u) -> bool {
-                const int st = u % NSTAGE;
-                if (!wait_bounded(&bars->v_full[st], (u / NSTAGE) & 1, ctl)) return false;
-                if (!wait_bounded(&bars->p_full, u & 1, ctl)) return false;
+        // Warp 9 + x issues query tile x's MMAs.  The whole warp runs the
+        // schedule (waits, descriptor arithmetic) in lock step, so operands
+        // are warp-uniform; lane 0 alone issues MMAs and commits.  Both
+        // issuers walk every key tile and commit the stage releases for each
+        // (no MMAs when their tile does not use it), so each phase of the
+        // two-arrival k_empty / v_empty barriers gets exactly one commit from
+        // each, in order.
+        const int x = warp - 9;
+        constexpr uint32_t idesc_pv = umma_idesc_bf16(BM, D, 0, 1);
+        // descriptors are built once; a k-step or stage only adds a constant
+        // to the 14-bit start-address field (addresses < 2^18)
+        const uint64_t dq = umma_smem_desc(smem_u32(sQ) + x * C::QTILE, 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dk0 = umma_smem_desc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dv0 = umma_smem_desc(smem_u32(sV), C::KCH, 8 * C::RB, C::LAYOUT);
+        const QTile q = x ? w.q[1] : w.q[0];
+        const int n_band = w.n_band;
+        const bool leader = lane == 0;
+        bool ok = warp_wait_bounded(&bars->q_full, 0, ctl);
+        auto pv_step = [&](int u) -> bool {
+            const int st = u % NSTAGE;
+            if (!warp_wait_bounded(&bars->v_full[st], (u / NSTAGE) & 1, ctl)) return false;
+            if (tile_active(q, n_band, u)) {
+                const int nk = tile_cols(w, a, u) / 16;
+                const uint64_t dv = dv0 + (uint64_t)((st * C::KTILE) >> 4);
+                const int c = tile_count(q, n_band, u), b = c & 1;
+                if (!warp_wait_bounded(&bars->p_full[x][b], (c >> 1) & 1, ctl)) return false;
                 tc_fence_after();
-                const uint32_t vb = v_base + st * C::TILE;
+                const uint32_t d_o = tmem + col_o(x), a_p = tmem + col_s(x, b);
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t da = umma_smem_desc(p_base + (kk / 4) * (BM * 128) + (kk % 4) * 32, 16, 1024,
-                                                       UMMA_SW128);
-                    const uint64_t db = umma_smem_desc(vb + kk * 16 * C::RB, C::CH_BYTES, 8 * C::RB, C::LAYOUT);
-                    mma_bf16_ss(tmem + C::COL_O, da, db, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        if (kk < nk)
+                            mma_bf16_ts(d_o, a_p + kk * 8, dv + (uint64_t)((kk * 16 * C::RB) >> 4), idesc_pv,
+                                        (c > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bars->pv_done[x][b]);
                 }
-                mma_commit(&bars->v_empty[st]);
-                mma_commit(&bars->pv_done);
-                return true;
-            };
-            for (int t = 0; t < w.n_tiles && ok; ++t) {
-                const int st = t % NSTAGE;
-                ok = wait_bounded(&bars->k_full[st], (t / NSTAGE) & 1, ctl);
+            }
+            if (leader) mma_commit(&bars->v_empty[st]);
+            __syncwarp();
+            return true;
+        };
+        for (int t = 0; t < w.n_tiles && ok; ++t) {
+            const int st = t % NSTAGE;
+            ok = warp_wait_bounded(&bars->k_full[st], (t / NSTAGE) & 1, ctl);
+            if (!ok) break;
+            if (tile_active(q, n_band, t)) {
+                const int c = tile_count(q, n_band, t), b = c & 1;
+                // S[x][b] holds P of this tile's predecessor in the buffer
+                // until that PV completes
+                if (c >= 2) ok = warp_wait_bounded(&bars->pv_done[x][b], ((c >> 1) - 1) & 1, ctl);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t kb = k_base + st * C::TILE;
-                const uint32_t d_s = tmem + C::COL_S + (t & 1) * BN;
+                const uint32_t idesc_qk = umma_idesc_bf16(BM, tile_cols(w, a, t), 0, 0);
+                const uint64_t dk = dk0 + (uint64_t)((st * C::KTILE) >> 4);
+                const uint32_t d_s = tmem + col_s(x, b);
+                if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int byte = kk * 32;
-                    const uint32_t off = (byte / C::RB) * C::CH_BYTES + (byte % C::RB);
-                    const uint64_t da = umma_smem_desc(q_base + off, 16, 8 * C::RB, C::LAYOUT);
-                    const uint64_t db = umma_smem_desc(kb + off, 16, 8 * C::RB, C::LAYOUT);
-                    mma_bf16_ss(d_s, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int byte = kk * 32;
+                        const uint64_t qo = (uint64_t)(((byte / C::RB) * C::QCH + (byte % C::RB)) >> 4);
+                        const uint64_t ko = (uint64_t)(((byte / C::RB) * C::KCH + (byte % C::RB)) >> 4);
+                        mma_bf16_ss(d_s, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bars->s_full[x][b]);
                 }
-                mma_commit(&bars->s_full[t & 1]);
-                mma_commit(&bars->k_empty[st]);
-                if (t >= 1) ok = issue_pv(t - 1);
             }
-            if (ok && w.n_tiles > 0) ok = issue_pv(w.n_tiles - 1);
-            // all MMAs this thread issued are complete before TMEM is freed
-            mma_commit(&bars->drain);
-            drain_wait(&bars->drain, 0, a.ctl.limit_ns);
+            if (leader) mma_commit(&bars->k_empty[st]);
+            __syncwarp();
+            if (t >= 1) ok = pv_step(t - 1);
+        }
+        if (ok && w.n_tiles > 0) ok = pv_step(w.n_tiles - 1);
+        // all MMAs lane 0 issued are complete before TMEM is freed
+        if (leader) {
+            mma_commit(&bars->drain[x]);
+            drain_wait(&bars->drain[x], 0, a.ctl.limit_ns);
         }
         __syncwarp();
     } else {
         // ------------------------------------------- softmax + epilogue --
-        const int r = threadIdx.x;              // row in tile = TMEM lane
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const int x = warp / 4;                 // query tile of this warpgroup
+        const int quarter = warp % 4;
+        const int r = quarter * 32 + lane;      // row in tile = TMEM lane
+        const QTile qt = x ? w.q[1] : w.q[0];
+        const int n_band = w.n_band;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         long long i_row;                        // absolute query position
-        if (w.mode == 0) i_row = w.m0 + r;
-        else i_row = (r < w.nrows) ? gb[w.gt * BM + r] : 0;
-        const bool row_real = r < w.nrows;
+        if (w.mode == 0) i_row = qt.m0 + r;
+        else i_row = (qt.active && r < qt.nrows) ? gb[qt.gt * BM + r] : 0;
+        const bool row_real = qt.active && r < qt.nrows;
+        const bool warp_has_rows = qt.active && quarter * 32 < qt.nrows;
+        const long long wi0 = (long long)qt.m0 + quarter * 32, wi1 = wi0 + 31;
         float m = -CUDART_INF_F, l = 0.f;
         bool ok = true;
-        float s[BN];
-        for (int t = 0; t < w.n_tiles; ++t) {
-            ok = warp_wait_bounded(&bars->s_full[t & 1], (t / 2) & 1, ctl);
+        for (int t = 0; t < w.n_tiles && qt.active; ++t) {
+            if (!tile_active(qt, n_band, t)) continue;
+            const int c = tile_count(qt, n_band, t), b = c & 1;
+            ok = warp_wait_bounded(&bars->s_full[x][b], (c >> 1) & 1, ctl);
             if (!ok) break;
             tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + C::COL_S + (t & 1) * BN + c * 32, s + c * 32);
-            tmem_ld_wait();
 
-            // ---- mask (edge tiles only) ----
-            if (w.mode == 1) {
-                const int key0 = t * BN;
-                if (key0 + BN > a.T) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (key0 + c >= a.T) s[c] = -CUDART_INF_F;
-                }
-            } else if (t < w.n_band) {
-                const int key0 = (w.j_lo + t) * BN;
-                const bool interior = (key0 + BN - 1 < a.T) && band_contains(w.m0 + BM - 1, key0, a.left, a.right) &&
-                                      band_contains(w.m0, key0 + BN - 1, a.left, a.right);
-                if (!interior) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const long long key = key0 + c;
-                        if (!(key < a.T && band_contains(i_row, key, a.left, a.right))) s[c] = -CUDART_INF_F;
+            // ---- which 32-key chunks can any row of this warp see ----
+            const bool band = t < w.n_band;
+            const int key0 = (w.j_lo + t) * BN;
+            int c_lo = 0, c_hi = -1;
+            bool interior = false;
+            if (warp_has_rows) {
+                if (w.mode == 1) {
+                    c_hi = (min(key0 + BN - 1, a.T - 1) - key0) / 32;
+                    interior = key0 + BN <= a.T;
+                } else if (band) {
+                    const long long lo = max(max((long long)key0, wi0 - a.left), 0LL);
+                    const long long hi = min(min((long long)key0 + BN - 1, wi1 + a.right), (long long)a.T - 1);
+                    if (lo <= hi) {
+                        c_lo = (int)((lo - key0) / 32);
+                        c_hi = (int)((hi - key0) / 32);
                     }
-                }
-            } else {
-                // gathered global keys: only those outside this row's band
-                const int c0 = (t - w.n_band) * BN;
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const int gc = c0 + c;
-                    bool keep = false;
-                    if (gc < a.g) keep = !band_contains(i_row, __ldg(gb + gc), a.left, a.right);
-                    if (!keep) s[c] = -CUDART_INF_F;
+                    interior = (key0 + BN - 1 < a.T) && band_contains(wi1, key0, a.left, a.right) &&
+                               band_contains(wi0, key0 + BN - 1, a.left, a.right);
+                } else {
+                    c_hi = (min(BN, a.g - (t - w.n_band) * BN) - 1) / 32;
                 }
             }
-
-            // ---- online softmax (log2 domain, lazy rescale) ----
-            // row max: 8 independent 3-input max chains, then a short tree
-            float mx8[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mx8[j] = fmax3(s[j], s[8 + j], s[16 + j]);
-#pragma unroll
-            for (int c = 24; c + 16 <= BN; c += 16)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx8[j] = fmax3(mx8[j], s[c + j], s[c + 8 + j]);
-#pragma unroll
-            for (int c = 24 + ((BN - 24) / 16) * 16; c < BN; c += 8)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(mx8[j], s[c + j]);
-            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                   fmaxf(mx8[6], mx8[7]));
-            const float mt = mx * a.scale_log2;
-            bool rescale_o = false;
-            float alpha = 1.f;
-            if (mt > m + RESCALE_LOG2) {
-                alpha = ex2_approx(m - mt);     // 0 when m was -inf
-                l *= alpha;
-                rescale_o = (t > 0);
-                m = mt;
+            // visible columns of this row as one int range (band, dense)
+            TileCtx k;
+            k.s_addr = tmem + lane_off + col_s(x, b);
+            k.c_lo = c_lo;
+            k.c_hi = c_hi;
+            k.col_lo = 0;
+            k.col_hi = BN - 1;
+            k.by_range = (w.mode == 1) || band;
+            if (w.mode == 1) {
+                k.col_hi = min(BN - 1, a.T - 1 - key0);
+            } else if (band) {
+                k.col_lo = (int)max(i_row - a.left - key0, 0LL);
+                k.col_hi = (int)min(min(i_row + a.right, (long long)a.T - 1) - key0, (long long)BN - 1);
             }
-            const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
-            // exponent arguments two at a time (fma.f32x2), four partial sums
-            const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-            const float2 nm2 = make_float2(-m_use, -m_use);
-            float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
-#pragma unroll
-            for (int c = 0; c < BN; c += 2) {
-                float2 x = fma2(make_float2(s[c], s[c + 1]), sc2, nm2);
-                s[c] = ex2_approx(x.x);
-                s[c + 1] = ex2_approx(x.y);
-                rs2[(c / 2) & 3] = add2(rs2[(c / 2) & 3], make_float2(s[c], s[c + 1]));
-            }
-            const float2 r01 = add2(rs2[0], rs2[1]), r23 = add2(rs2[2], rs2[3]);
-            const float2 rsum = add2(r01, r23);
-            l += rsum.x + rsum.y;
+            k.gc_base = (t - w.n_band) * BN;
+            k.i_row = i_row;
+            bool rescale_o;
+            float alpha;
+            if (interior && c_lo == 0 && c_hi == BN / 32 - 1)
+                softmax_tile<true>(k, a, gb, m, l, rescale_o, alpha, c == 0);
+            else
+                softmax_tile<false>(k, a, gb, m, l, rescale_o, alpha, c == 0);
 
-            // PV of the previous tile must be done: it reads the P buffer and
-            // writes O, which a rescale touches
-            if (t > 0) {
-                ok = warp_wait_bounded(&bars->pv_done, (t - 1) & 1, ctl);
+            // O rescale (rare): wait for the previous tile's PV, which
+            // accumulates into O; this tile's PV waits for P
+            if (__any_sync(0xffffffffu, rescale_o)) {
+                const int cp = c - 1, bp = cp & 1;
+                ok = warp_wait_bounded(&bars->pv_done[x][bp], (cp >> 1) & 1, ctl);
                 if (!ok) break;
                 tc_fence_after();
-            }
-            if (__any_sync(0xffffffffu, rescale_o)) {
+                const float f = rescale_o ? alpha : 1.f;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float ov[32];
-                    tmem_ld32(lane_base + C::COL_O + c * 32, ov);
-                    tmem_ld_wait();
-                    const float f = rescale_o ? alpha : 1.f;
+                for (int cc = 0; cc < D / 16; ++cc) {
+                    float ov[16];
+                    tmem_ld16(tmem + lane_off + col_o(x) + cc * 16, ov);
+                    tmem_ld_wait_dep16(ov);
+                    uint32_t ou[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] *= f;
-                    tmem_st32(lane_base + C::COL_O + c * 32, ov);
+                    for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(ov[e] * f);
+                    tmem_st16u(tmem + lane_off + col_o(x) + cc * 16, ou);
                 }
-                tmem_st_wait();
             }
-            // P (bf16) into the swizzled K-major A-operand tile
-#pragma unroll
-            for (int u = 0; u < BN / 8; ++u) {
-                uint4 pk;
-                pk.x = pack_bf16x2(s[u * 8 + 0], s[u * 8 + 1]);
-                pk.y = pack_bf16x2(s[u * 8 + 2], s[u * 8 + 3]);
-                pk.z = pack_bf16x2(s[u * 8 + 4], s[u * 8 + 5]);
-                pk.w = pack_bf16x2(s[u * 8 + 6], s[u * 8 + 7]);
-                const int kc = u / 8, g16 = u % 8;
-                *reinterpret_cast<uint4 *>(sP + kc * (BM * 128) + r * 128 + ((g16 ^ (r & 7)) << 4)) = pk;
-            }
-            fence_proxy_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full);
+            if (lane == 0) mbar_arrive(&bars->p_full[x][b]);
         }
 
         // ---- epilogue ----
-        if (ok && w.n_tiles > 0) ok = warp_wait_bounded(&bars->pv_done, (w.n_tiles - 1) & 1, ctl);
-        if (ok) {
+        const int nx = tiles_of(qt, w.n_glob);
+        if (ok && nx > 0) {
+            const int cl = nx - 1;
+            ok = warp_wait_bounded(&bars->pv_done[x][cl & 1], (cl >> 1) & 1, ctl);
+        }
+        const bool direct = (w.mode == 1) || (a.gidx != nullptr && a.g > 0);
+        uint8_t *stage = sQ + x * C::QTILE;
+        if (ok && qt.active) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
-            const bool direct = (w.mode == 1) || (a.gidx != nullptr && a.g > 0);
             __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
             bool skip_row = !row_real;
             if (w.mode == 0 && direct && row_real) {
@@ -489,42 +687,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 skip_row = (lo < a.g && gb[lo] == i_row);
             }
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float ov[32];
-                tmem_ld32(lane_base + C::COL_O + c * 32, ov);
-                tmem_ld_wait();
+            for (int cc = 0; cc < D / 16; ++cc) {
+                float ov[16];
+                tmem_ld16(tmem + lane_off + col_o(x) + cc * 16, ov);
+                tmem_ld_wait_dep16(ov);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     uint4 pk;
                     pk.x = pack_bf16x2(ov[u * 8 + 0] * inv, ov[u * 8 + 1] * inv);
                     pk.y = pack_bf16x2(ov[u * 8 + 2] * inv, ov[u * 8 + 3] * inv);
                     pk.z = pack_bf16x2(ov[u * 8 + 4] * inv, ov[u * 8 + 5] * inv);
                     pk.w = pack_bf16x2(ov[u * 8 + 6] * inv, ov[u * 8 + 7] * inv);
-                    const int e = c * 32 + u * 8;
+                    const int e = cc * 16 + u * 8;
                     if (direct) {
                         if (!skip_row) {
-                            __nv_bfloat16 *dst = o + (((long long)w.b * a.T + i_row) * a.Hq + w.h) * D + e;
+                            __nv_bfloat16 *dst = o + (((long long)w.b * a.T + i_row) * a.Hq + qt.h) * D + e;
                             *reinterpret_cast<uint4 *>(dst) = pk;
                         }
                     } else {
-                        *reinterpret_cast<uint4 *>(sQ + tile_offset<D>(r, e)) = pk;
+                        *reinterpret_cast<uint4 *>(stage + tile_offset<D>(r, e, C::QCH)) = pk;
                     }
                 }
             }
             if (a.lse && row_real && !skip_row)
-                a.lse[((long long)w.b * a.Hq + w.h) * a.T + i_row] =
+                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_row] =
                     (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
-        // staging tile complete -> one thread stores it (bounded; an abort
-        // anywhere in the CTA skips the store)
-        const bool direct_store = (w.mode == 1) || (a.gidx != nullptr && a.g > 0);
-        if (!direct_store) {
+        // staging tile complete -> one thread per warpgroup stores it
+        // (bounded; an abort anywhere in the CTA skips the store)
+        if (!direct && qt.active) {
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->epi);
-            if (r == 0 && wait_bounded(&bars->epi, 0, ctl) && !bars->abort) {
+            if (lane == 0) mbar_arrive(&bars->epi[x]);
+            if (r == 0 && wait_bounded(&bars->epi[x], 0, ctl) && !bars->abort) {
                 for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_store_4d(&tmO, sQ + ch * C::CH_BYTES, ch * C::E, w.h, w.m0, w.b);
+                    tma_store_4d(&tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
                 tma_store_commit();
                 tma_store_wait_all();
             }
@@ -533,7 +730,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -558,17 +755,17 @@ EncodeTiledFn get_encode()
     return fn;
 }
 
-// [B,T,H,D] bf16 viewed as a 4-D tensor (D, H, T, B); box = one chunk of 128
-// rows of one head.
+// [B,T,H,D] bf16 viewed as a 4-D tensor (D, H, T, B); box = one chunk of
+// `rows` rows of one head.
 template <int D>
-bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H)
+bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int rows)
 {
     using C = Cfg<D>;
     EncodeTiledFn enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    cuuint32_t box[4] = {(cuuint32_t)C::E, 1, 128, 1};
+    cuuint32_t box[4] = {(cuuint32_t)C::E, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -582,8 +779,8 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
 {
     using C = Cfg<D>;
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map<D>(&mq, a.q, a.B, a.T, a.Hq) || !make_map<D>(&mk, a.k, a.B, a.T, a.Hkv) ||
-        !make_map<D>(&mv, a.v, a.B, a.T, a.Hkv) || !make_map<D>(&mo, a.o, a.B, a.T, a.Hq))
+    if (!make_map<D>(&mq, a.q, a.B, a.T, a.Hq, BM) || !make_map<D>(&mk, a.k, a.B, a.T, a.Hkv, BN) ||
+        !make_map<D>(&mv, a.v, a.B, a.T, a.Hkv, BN) || !make_map<D>(&mo, a.o, a.B, a.T, a.Hq, BM))
         return cudaErrorInvalidValue;
     static bool attr_set[64] = {};
     int dev = 0;
@@ -594,14 +791,21 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
+    const int G = a.Hq / a.Hkv;
+    const bool pair_heads = (G % 2) == 0;
     const int nqt = (a.T + BM - 1) / BM;
+    const int ngt = (a.g + BM - 1) / BM;
     const bool globals = a.gidx != nullptr && a.g > 0;
+    // CTAs: pairs of heads (even group size) or pairs of row tiles / global
+    // row groups of one head
+    const int units_q = pair_heads ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2);
+    const int units_g = pair_heads ? (a.Hq / 2) * ngt : a.Hq * ((ngt + 1) / 2);
     int n_mode1 = 0, n_mode0 = 0;
     if (mode == 0) {
-        n_mode0 = a.B * a.Hq * nqt;
-        if (globals) n_mode1 = a.B * a.Hq * ((a.g + BM - 1) / BM);
+        n_mode0 = a.B * units_q;
+        if (globals) n_mode1 = a.B * units_g;
     } else {
-        n_mode1 = a.B * a.Hq * ((a.g + BM - 1) / BM);
+        n_mode1 = a.B * units_g;
     }
     const int grid = n_mode0 + n_mode1;
     if (grid == 0) return cudaSuccess;
