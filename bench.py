@@ -319,7 +319,7 @@ def gpu_arm(args, world, rank, local):
                      "achieved": round(pre_tf, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(pre_tf / peak_t, 4), "peak_source": peak_src + " bf16 burst",
                      "traffic": recorded_traffic("prefill_mistral")},
-        "roofline_decode": {"kernel": "decode_kernel<bf16,128,4> + combine", "bound": "hbm",
+        "roofline_decode": {"kernel": "decode_bf16_kernel<128,4> + combine", "bound": "hbm",
                             "achieved": round(dec_gbs, 1), "peak": peak_h, "unit": "GB/s",
                             "frac": round(dec_gbs / peak_h, 4), "peak_source": peak_src + " copy",
                             "traffic": recorded_traffic("decode_mistral")},
