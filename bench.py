@@ -89,9 +89,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# the sources each recorded kernel is built from
+KERNEL_SOURCES = {
+    "prefill_mistral": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h"),
+    "longformer": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h"),
+    "decode_mistral": ("simt_kernels.cu", "ptx.cuh", "swa_internal.h"),
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
-    for f in ("prefill_tc.cu", "simt_kernels.cu", "ptx.cuh", "swa_internal.h"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "decode_swa_prefill_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -99,14 +107,14 @@ def kernel_source_hash():
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch from a committed ncu summary, only if it was taken
-    on the current kernel sources."""
+    on the kernel's current sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -41,9 +41,9 @@
 // The running max is only raised when a tile's max exceeds it by more than
 // 2^8; P then stays <= 256 and O, l share one reference, so the final O/l is
 // exact; raising it rescales l and the O row in TMEM.  Per warp, 32-key
-// chunks that no row of the warp can see are skipped.  Half of the
-// exponentials run on the MUFU (ex2.approx), half as a range-reduced cubic on
-// the FMA pipe (exp2_poly2), which roughly halves the MUFU time per tile.
+// chunks that no row of the warp can see are skipped.  Three quarters of the
+// exponentials run on the MUFU (ex2.approx), one quarter as a range-reduced
+// cubic on the FMA pipe (exp2_poly2), which shortens the MUFU time per tile.
 //
 // Every mbarrier wait is bounded (wait_bounded): on expiry the CTA records
 // SWA_STATUS_TIMEOUT, drains its own in-flight copies and MMAs with a second
@@ -118,6 +118,7 @@ struct Bars {
     uint64_t pv_done[2][2];  // [tile][buffer]
     uint64_t drain[2];
     uint64_t epi[2];
+    uint64_t a_first;        // tile A's first QK^T complete (used once)
     uint32_t tmem_base;
     int abort;
 };
@@ -401,6 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(&bars->epi[x], BM / 32);
             mbar_init(&bars->drain[x], 1);
         }
+        mbar_init(&bars->a_first, 1);
         bars->abort = 0;
         fence_mbar_init();
     }
@@ -511,6 +513,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int n_band = w.n_band;
         const bool leader = lane == 0;
         bool ok = warp_wait_bounded(&bars->q_full, 0, ctl);
+        // Tile B starts once tile A's first QK^T has completed: the two
+        // tiles then run half a step apart, so one tile's MMAs tend to fill
+        // the tensor core while the other waits for its softmax.
+        const bool offset_b = w.q[0].active && tile_active(w.q[0], n_band, 0);
+        if (ok && x == 1 && offset_b) ok = warp_wait_bounded(&bars->a_first, 0, ctl);
         auto pv_step = [&](int u) -> bool {
             const int st = u % NSTAGE;
             if (!warp_wait_bounded(&bars->v_full[st], (u / NSTAGE) & 1, ctl)) return false;
@@ -557,6 +564,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         mma_bf16_ss(d_s, dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&bars->s_full[x][b]);
+                    if (x == 0 && t == 0) mma_commit(&bars->a_first);
                 }
             }
             if (leader) mma_commit(&bars->k_empty[st]);
