@@ -51,6 +51,9 @@ def _load():
         lib.oracle_swa_decode.argtypes = [p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
                                           c_double]
         lib.oracle_swa_decode.restype = c_int
+        lib.oracle_swa_prefill_chunk.argtypes = [p, p, p, p, p, p, p, p, c_long, c_long, c_long, c_long,
+                                                 c_long, c_long, c_double]
+        lib.oracle_swa_prefill_chunk.restype = c_int
         _lib = lib
     return _lib
 
@@ -198,4 +201,23 @@ def swa_decode(q, k_cache, v_cache, pos, scale=None):
     o = np.zeros((B, Hq, d)); lse = np.zeros((B, Hq))
     _load().oracle_swa_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(_i32(pos)), _ptr(o), _ptr(lse),
                               B, Hq, Hkv, d, W, float(scale))
+    return o, lse
+
+
+def swa_prefill_chunk(q, k, v, k_cache, v_cache, pos, scale=None):
+    """Causal prefill of a chunk of n tokens at positions pos[b].. that reads
+    the keys before pos[b] from the W-slot ring (Ultralytics ring-buffer
+    paragraph; robocikowo.com opening definition).  q [B,n,Hq,d], k/v
+    [B,n,Hkv,d], caches [B,Hkv,W,d] not yet holding the chunk, pos [B].
+    Returns o [B,n,Hq,d], lse [B,Hq,n]."""
+    q, k, v, kc, vc = _f64(q), _f64(k), _f64(v), _f64(k_cache), _f64(v_cache)
+    B, n, Hq, d = q.shape
+    Hkv, W = kc.shape[1], kc.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, n, Hq, d)); lse = np.zeros((B, Hq, n))
+    rc = _load().oracle_swa_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc), _ptr(_i32(pos)),
+                                          _ptr(o), _ptr(lse), B, n, Hq, Hkv, d, W, float(scale))
+    if rc != 0:
+        raise ValueError("negative position")
     return o, lse

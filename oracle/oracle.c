@@ -295,3 +295,53 @@ int oracle_swa_decode(const double *q, const double *kc, const double *vc, const
     free(kr); free(vr); free(s);
     return 0;
 }
+
+/* ---------------------------------------------------------- chunk prefill -- */
+
+/* Prefill of n new tokens at positions pos[b] .. pos[b]+n-1 that continue a
+ * sequence whose earlier tokens live in the W-slot ring [P4 ring-buffer
+ * paragraph: position p sits in slot p mod W and only the latest W tokens
+ * are kept; P3 opening definition: query P sees the keys at positions
+ * P-W+1 .. P].  Keys at positions >= pos[b] are rows of the chunk itself;
+ * earlier ones are read from ring slot (position mod W), which holds them as
+ * long as the chunk has not been appended yet.  Keys in list order of
+ * position.  q/o [B,n,Hq,d]; k/v [B,n,Hkv,d]; caches [B,Hkv,W,d];
+ * lse (nullable) [B,Hq,n].  Returns -1 for a negative position. */
+int oracle_swa_prefill_chunk(const double *q, const double *k, const double *v, const double *kc,
+                             const double *vc, const int32_t *pos, double *o, double *lse, long B, long n,
+                             long Hq, long Hkv, long d, long W, double scale)
+{
+    for (long b = 0; b < B; b++)
+        if (pos[b] < 0) return -1;
+    const double **kr = malloc(sizeof(double *) * (size_t)W);
+    const double **vr = malloc(sizeof(double *) * (size_t)W);
+    double *s = malloc(sizeof(double) * (size_t)W);
+    for (long b = 0; b < B; b++) {
+        const long p0 = pos[b];
+        for (long h = 0; h < Hq; h++) {
+            const long hk = h * Hkv / Hq;
+            for (long t = 0; t < n; t++) {
+                const long P = p0 + t;
+                const long lo = P - W + 1 > 0 ? P - W + 1 : 0;
+                long nk = 0;
+                for (long j = lo; j <= P; j++) {
+                    if (j >= p0) {
+                        kr[nk] = k + ((b * n + (j - p0)) * Hkv + hk) * d;
+                        vr[nk] = v + ((b * n + (j - p0)) * Hkv + hk) * d;
+                    } else {
+                        const long sl = oracle_slot(j, W);
+                        kr[nk] = kc + ((b * Hkv + hk) * W + sl) * d;
+                        vr[nk] = vc + ((b * Hkv + hk) * W + sl) * d;
+                    }
+                    nk++;
+                }
+                double l;
+                attend_row(q + ((b * n + t) * Hq + h) * d, kr, vr, nk, d, scale, o + ((b * n + t) * Hq + h) * d,
+                           &l, s);
+                if (lse) lse[(b * Hq + h) * n + t] = l;
+            }
+        }
+    }
+    free(kr); free(vr); free(s);
+    return 0;
+}
