@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "SwaError", "load", "library_path", "EXPORTED",
-    "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
+    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode",
     "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
     "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
@@ -29,7 +29,7 @@ SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 
 # every symbol include/swa.h declares
 EXPORTED = [
-    "swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode_workspace_bytes",
+    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
     "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
@@ -55,6 +55,7 @@ def load():
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.swa_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.swa_prefill_global.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -67,7 +68,7 @@ def load():
     lib.swa_set_wait_limit_ns.restype = None
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
-    for name in ("swa_prefill", "swa_prefill_global", "swa_cache_append", "swa_decode",
+    for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -124,6 +125,26 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
     st = load().swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
                             float(scale), _dtype_code(q), _stream(stream))
     _check(st, "swa_prefill")
+    return o
+
+
+def swa_prefill_chunk(q, k, v, k_cache, v_cache, pos, scale=None, o=None, lse=None, stream=None):
+    """Causal prefill of a chunk q/k/v [B,n,H,d] at positions pos[b].. (int32
+    [B]) that reads earlier keys from the rings k_cache/v_cache [B,Hkv,W,d]
+    (not yet holding the chunk); returns o (and fills lse [B,Hq,n])."""
+    _dev_contig(q, k, v, o, lse, k_cache, v_cache, pos)
+    B, n, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, n, Hkv, d) and v.shape == k.shape, "k/v shape")
+    W = k_cache.shape[2]
+    _need(k_cache.shape == (B, Hkv, W, d) and v_cache.shape == k_cache.shape, "cache shape")
+    _need(pos.dtype == torch.int32 and pos.shape == (B,), "pos [B] int32")
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(pos), B, n, Hq, Hkv, d, W, float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_prefill_chunk")
     return o
 
 

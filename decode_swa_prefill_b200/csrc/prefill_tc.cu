@@ -151,6 +151,8 @@ struct Work {
     int n_band;   // band key tiles streamed by TMA
     int n_glob;   // gathered tiles of global keys (band mode with globals)
     int n_tiles;
+    long long p0;   // position of query row 0 (a chunk continuing a ring; else 0)
+    long long kend; // one past the last key position (p0 + T)
 };
 
 // Does query tile q use key tile t, and which of its tiles is it?
@@ -197,6 +199,8 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, int n_mode1)
         w.j_lo = 0;
         w.n_band = nkt;
         w.n_glob = 0;
+        w.p0 = 0;
+        w.kend = a.T;
     } else {
         bid -= n_mode1;
         w.mode = 0;
@@ -216,21 +220,26 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, int n_mode1)
                 if (qt < nqt) w.q[x] = QTile{h, qt * BM, 0, min(BM, a.T - qt * BM), 0, 0, true};
             }
         }
-        int lo = a.T, hi = -1;
-        int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+        // a chunk continuing a ring starts at position pos[b] (a negative
+        // entry is read as 0; the producer records it)
+        const long long p0 = a.pos ? max((long long)a.pos[w.b], 0LL) : 0LL;
+        w.p0 = p0;
+        w.kend = p0 + a.T;
+        long long lo = w.kend, hi = -1;
+        long long lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
         for (int x = 0; x < 2; ++x) {
             if (!w.q[x].active) continue;
-            lo_x[x] = max(0, w.q[x].m0 - a.left);
-            hi_x[x] = min(a.T - 1, w.q[x].m0 + BM - 1 + a.right);
+            lo_x[x] = max(0LL, p0 + w.q[x].m0 - a.left);
+            hi_x[x] = min(w.kend - 1, p0 + w.q[x].m0 + BM - 1 + a.right);
             lo = min(lo, lo_x[x]);
             hi = max(hi, hi_x[x]);
         }
-        w.j_lo = lo / BN;
-        w.n_band = hi / BN - w.j_lo + 1;
+        w.j_lo = (int)(lo / BN);
+        w.n_band = (int)(hi / BN) - w.j_lo + 1;
         for (int x = 0; x < 2; ++x)
             if (w.q[x].active) {
-                w.q[x].ts = lo_x[x] / BN - w.j_lo;
-                w.q[x].te = hi_x[x] / BN - w.j_lo + 1;
+                w.q[x].ts = (int)(lo_x[x] / BN) - w.j_lo;
+                w.q[x].te = (int)(hi_x[x] / BN) - w.j_lo + 1;
             }
         w.n_glob = (a.gidx != nullptr && a.g > 0) ? (a.g + BN - 1) / BN : 0;
     }
@@ -262,6 +271,22 @@ __device__ __forceinline__ void gather_tile(uint8_t *dst, int rows, int ch_bytes
         const long long pos = r < nrows ? rows_idx[r] : 0;
         const __nv_bfloat16 *src = base + (((long long)b * T + pos) * H + head) * D + u * 8;
         cp_async16(dst + tile_offset<D>(r, u * 8, ch_bytes), src, r < nrows ? 16u : 0u);
+    }
+    cp_async_wait_all();
+}
+
+// Producer-warp gather of `rows` rows into a swizzled tile with 16-byte
+// cp.async copies; row_src(r) gives row r's source, or null for zeros.  All
+// 32 lanes.
+template <int D, typename RowSrc>
+__device__ __forceinline__ void gather_rows(uint8_t *dst, int rows, int ch_bytes, const __nv_bfloat16 *any_valid,
+                                            int lane, RowSrc row_src)
+{
+    constexpr int GR = D / 8; // 16-byte granules per row
+    for (int idx = lane; idx < rows * GR; idx += 32) {
+        const int r = idx / GR, u = idx % GR;
+        const __nv_bfloat16 *src = row_src(r);
+        cp_async16(dst + tile_offset<D>(r, u * 8, ch_bytes), src ? src + u * 8 : any_valid, src ? 16u : 0u);
     }
     cp_async_wait_all();
 }
@@ -370,6 +395,7 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                          const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
                           const TcPrefillArgs a, const int n_mode1)
 {
     using C = Cfg<D>;
@@ -444,46 +470,60 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->q_full);
         }
+        if (a.pos && lane == 0 && a.pos[w.b] < 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+        // One K or V key tile into stage st: a TMA tile of the key tensor or
+        // of the ring, or 16-byte cp.async row copies (global keys; ring rows
+        // that wrap around the ring's end or meet the chunk's first row).
+        auto load_tile = [&](bool is_v, int st, int t) {
+            uint8_t *dst = (is_v ? sV : sK) + st * C::KTILE;
+            uint64_t *bar = is_v ? &bars->v_full[st] : &bars->k_full[st];
+            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(is_v ? a.v : a.k);
+            if (t >= w.n_band) {
+                const int gt = t - w.n_band;
+                gather_tile<D>(dst, BN, C::KCH, src, gb + gt * BN, min(BN, a.g - gt * BN), w.b, a.T, a.Hkv, w.hk,
+                               lane);
+            } else {
+                const long long key0 = (long long)(w.j_lo + t) * BN;
+                const bool ring_tile = a.pos && key0 < w.p0;
+                const long long slot0 = ring_tile ? key0 % a.W_ring : 0;
+                if (!ring_tile || (key0 + BN <= w.p0 && slot0 + BN <= a.W_ring)) {
+                    if (lane == 0) {
+                        mbar_expect_tx(bar, C::KTILE);
+                        for (int ch = 0; ch < C::NCH; ++ch) {
+                            if (ring_tile)
+                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmVr : &tmKr, bar, ch * C::E, (int)slot0, w.hk,
+                                            w.b);
+                            else
+                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk,
+                                            (int)(key0 - w.p0), w.b);
+                        }
+                    }
+                    return;
+                }
+                const __nv_bfloat16 *ring = static_cast<const __nv_bfloat16 *>(is_v ? a.vc : a.kc);
+                gather_rows<D>(dst, BN, C::KCH, src, lane, [&](int r) -> const __nv_bfloat16 * {
+                    const long long p = key0 + r;
+                    if (p >= w.p0) {
+                        const long long row = p - w.p0;
+                        return row < a.T ? src + (((long long)w.b * a.T + row) * a.Hkv + w.hk) * D : nullptr;
+                    }
+                    return ring + (((long long)w.b * a.Hkv + w.hk) * a.W_ring + p % a.W_ring) * D;
+                });
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
         for (int t = 0; t < w.n_tiles && ok; ++t) {
-            const bool band = t < w.n_band;
-            const int key0 = (w.j_lo + t) * BN;
-            const int gt = t - w.n_band;
-            const int nr = band ? 0 : min(BN, a.g - gt * BN);
             const int st = t % NSTAGE;
             const uint32_t par = ((t / NSTAGE) & 1) ^ 1;
             ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
             if (!ok) break;
-            if (band) {
-                if (lane == 0) {
-                    mbar_expect_tx(&bars->k_full[st], C::KTILE);
-                    for (int ch = 0; ch < C::NCH; ++ch)
-                        tma_load_4d(sK + st * C::KTILE + ch * C::KCH, &tmK, &bars->k_full[st], ch * C::E, w.hk,
-                                    key0, w.b);
-                }
-            } else {
-                gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
-                               gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->k_full[st]);
-            }
+            load_tile(false, st, t);
             kiss[st]++;
             ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
             if (!ok) break;
-            if (band) {
-                if (lane == 0) {
-                    mbar_expect_tx(&bars->v_full[st], C::KTILE);
-                    for (int ch = 0; ch < C::NCH; ++ch)
-                        tma_load_4d(sV + st * C::KTILE + ch * C::KCH, &tmV, &bars->v_full[st], ch * C::E, w.hk,
-                                    key0, w.b);
-                }
-            } else {
-                gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
-                               gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->v_full[st]);
-            }
+            load_tile(true, st, t);
             viss[st]++;
         }
         if (!ok && lane == 0) {
@@ -587,11 +627,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int n_band = w.n_band;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         long long i_row;                        // absolute query position
-        if (w.mode == 0) i_row = qt.m0 + r;
+        if (w.mode == 0) i_row = w.p0 + qt.m0 + r;
         else i_row = (qt.active && r < qt.nrows) ? gb[qt.gt * BM + r] : 0;
+        const long long i_out = i_row - w.p0;   // row in q / o / lse
         const bool row_real = qt.active && r < qt.nrows;
         const bool warp_has_rows = qt.active && quarter * 32 < qt.nrows;
-        const long long wi0 = (long long)qt.m0 + quarter * 32, wi1 = wi0 + 31;
+        const long long wi0 = w.p0 + qt.m0 + quarter * 32, wi1 = wi0 + 31;
         float m = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; t < w.n_tiles && qt.active; ++t) {
@@ -603,21 +644,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
             // ---- which 32-key chunks can any row of this warp see ----
             const bool band = t < w.n_band;
-            const int key0 = (w.j_lo + t) * BN;
+            const long long key0 = (long long)(w.j_lo + t) * BN;
             int c_lo = 0, c_hi = -1;
             bool interior = false;
             if (warp_has_rows) {
                 if (w.mode == 1) {
-                    c_hi = (min(key0 + BN - 1, a.T - 1) - key0) / 32;
-                    interior = key0 + BN <= a.T;
+                    c_hi = (int)((min(key0 + BN - 1, w.kend - 1) - key0) / 32);
+                    interior = key0 + BN <= w.kend;
                 } else if (band) {
-                    const long long lo = max(max((long long)key0, wi0 - a.left), 0LL);
-                    const long long hi = min(min((long long)key0 + BN - 1, wi1 + a.right), (long long)a.T - 1);
+                    const long long lo = max(max(key0, wi0 - a.left), 0LL);
+                    const long long hi = min(min(key0 + BN - 1, wi1 + a.right), w.kend - 1);
                     if (lo <= hi) {
                         c_lo = (int)((lo - key0) / 32);
                         c_hi = (int)((hi - key0) / 32);
                     }
-                    interior = (key0 + BN - 1 < a.T) && band_contains(wi1, key0, a.left, a.right) &&
+                    interior = (key0 + BN - 1 < w.kend) && band_contains(wi1, key0, a.left, a.right) &&
                                band_contains(wi0, key0 + BN - 1, a.left, a.right);
                 } else {
                     c_hi = (min(BN, a.g - (t - w.n_band) * BN) - 1) / 32;
@@ -632,10 +673,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             k.col_hi = BN - 1;
             k.by_range = (w.mode == 1) || band;
             if (w.mode == 1) {
-                k.col_hi = min(BN - 1, a.T - 1 - key0);
+                k.col_hi = (int)min((long long)BN - 1, w.kend - 1 - key0);
             } else if (band) {
                 k.col_lo = (int)max(i_row - a.left - key0, 0LL);
-                k.col_hi = (int)min(min(i_row + a.right, (long long)a.T - 1) - key0, (long long)BN - 1);
+                k.col_hi = (int)min(min(i_row + a.right, w.kend - 1) - key0, (long long)BN - 1);
             }
             k.gc_base = (t - w.n_band) * BN;
             k.i_row = i_row;
@@ -709,7 +750,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int e = cc * 16 + u * 8;
                     if (direct) {
                         if (!skip_row) {
-                            __nv_bfloat16 *dst = o + (((long long)w.b * a.T + i_row) * a.Hq + qt.h) * D + e;
+                            __nv_bfloat16 *dst = o + (((long long)w.b * a.T + i_out) * a.Hq + qt.h) * D + e;
                             *reinterpret_cast<uint4 *>(dst) = pk;
                         }
                     } else {
@@ -718,7 +759,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             if (a.lse && row_real && !skip_row)
-                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_row] =
+                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_out] =
                     (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
         // staging tile complete -> one thread per warpgroup stores it
@@ -782,14 +823,40 @@ bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int rows)
     return r == CUDA_SUCCESS;
 }
 
+// Ring cache [B,Hkv,W,D] bf16 viewed as (D, W, Hkv, B); box = one chunk of
+// BN consecutive slots of one kv head.
+template <int D>
+bool make_ring_map(CUtensorMap *m, const void *ptr, int B, int Hkv, int W)
+{
+    using C = Cfg<D>;
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)Hkv, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)W * D * 2, (cuuint64_t)Hkv * W * D * 2};
+    cuuint32_t box[4] = {(cuuint32_t)C::E, (cuuint32_t)BN, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     C::RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
 {
     using C = Cfg<D>;
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv, mo, mkr, mvr;
     if (!make_map<D>(&mq, a.q, a.B, a.T, a.Hq, BM) || !make_map<D>(&mk, a.k, a.B, a.T, a.Hkv, BN) ||
         !make_map<D>(&mv, a.v, a.B, a.T, a.Hkv, BN) || !make_map<D>(&mo, a.o, a.B, a.T, a.Hq, BM))
         return cudaErrorInvalidValue;
+    if (a.pos) {
+        if (!make_ring_map<D>(&mkr, a.kc, a.B, a.Hkv, a.W_ring) || !make_ring_map<D>(&mvr, a.vc, a.B, a.Hkv, a.W_ring))
+            return cudaErrorInvalidValue;
+    } else {
+        mkr = mk; // unused without a ring
+        mvr = mv;
+    }
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -817,7 +884,7 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
     }
     const int grid = n_mode0 + n_mode1;
     if (grid == 0) return cudaSuccess;
-    swa_prefill_tc_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, n_mode1);
+    swa_prefill_tc_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, n_mode1);
     return cudaGetLastError();
 }
 

@@ -105,9 +105,26 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
         acc[e] = 0.f;
     }
     float m = -CUDART_INF_F, l = 0.f;
+    // chunk continuing a ring: row i is at position p0 + i; positions below
+    // p0 are read from ring slot (position mod W_ring)
+    long long p0 = 0;
+    if (a.pos) {
+        p0 = a.pos[b];
+        if (p0 < 0) {
+            if (lane == 0 && i == 0 && h == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+            p0 = 0;
+        }
+    }
     auto visit = [&](long long j) {
-        const float *krow = a.k + (((long long)b * a.T + j) * a.Hkv + hk) * a.d;
-        const float *vrow = a.v + (((long long)b * a.T + j) * a.Hkv + hk) * a.d;
+        const float *krow, *vrow;
+        if (j >= p0) {
+            krow = a.k + (((long long)b * a.T + (j - p0)) * a.Hkv + hk) * a.d;
+            vrow = a.v + (((long long)b * a.T + (j - p0)) * a.Hkv + hk) * a.d;
+        } else {
+            const long long sl = j % a.W_ring;
+            krow = a.kc + (((long long)b * a.Hkv + hk) * a.W_ring + sl) * a.d;
+            vrow = a.vc + (((long long)b * a.Hkv + hk) * a.W_ring + sl) * a.d;
+        }
         float dot = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -131,8 +148,9 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
     if (row_global) {
         for (long long j = 0; j < a.T; ++j) visit(j);
     } else {
-        const long long lo = max(0LL, (long long)i - a.left);
-        const long long hi = min((long long)a.T - 1, (long long)i + a.right);
+        const long long ip = p0 + i;  // absolute position of the row
+        const long long lo = max(0LL, ip - a.left);
+        const long long hi = min(p0 + a.T - 1, ip + a.right);
         for (long long j = lo; j <= hi; ++j) visit(j);
         if (gb)
             for (int c = 0; c < a.g; ++c)

@@ -141,6 +141,37 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
     return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
 }
 
+swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *o, float *lse, const void *k_cache,
+                             const void *v_cache, const int32_t *pos, int B, int n, int Hq, int Hkv, int d, int W,
+                             float scale, swa_dtype dt, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, B, n, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK || B == 0 || n == 0) return st;
+    if (!k_cache || !v_cache || !pos) return SWA_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(pos, 4)) return SWA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == SWA_DTYPE_F32) {
+        swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(o), lse, B, n, Hq, Hkv, d, W - 1, 0,
+                              nullptr, 0, scale};
+        a.pos = pos;
+        a.kc = static_cast<const float *>(k_cache);
+        a.vc = static_cast<const float *>(v_cache);
+        a.W_ring = W;
+        if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+        return from_cuda(swa::launch_prefill_f32(a, s));
+    }
+    swa::TcPrefillArgs a{};
+    a.B = B; a.T = n; a.Hq = Hq; a.Hkv = Hkv;
+    a.left = W - 1; a.right = 0;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.lse = lse; a.gidx = nullptr; a.g = 0;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    a.pos = pos; a.kc = k_cache; a.vc = v_cache; a.W_ring = W;
+    if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+}
+
 swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new, const int32_t *pos,
                             int32_t *slot_out, int B, int n, int Hkv, int d, int W, swa_dtype dt, void *stream)
 {

@@ -34,6 +34,12 @@ struct TcPrefillArgs {
     int g;
     const void *q, *k, *v;    // raw pointers (gathers)
     void *o;                  // raw output pointer (scatter in global-row mode)
+    // chunk continuing a ring (band mode): T is the chunk length n, query row
+    // r of batch b is at position pos[b]+r; keys before pos[b] come from the
+    // W_ring-slot caches kc / vc [B,Hkv,W_ring,d]
+    const int32_t *pos;       // null: no ring
+    const void *kc, *vc;
+    int W_ring;
     DeviceCtl ctl;
 };
 
@@ -51,6 +57,11 @@ struct F32PrefillArgs {
     const int32_t *gidx;
     int g;
     float scale;
+    // chunk continuing a ring (causal only), as in TcPrefillArgs
+    const int32_t *pos;
+    const float *kc, *vc;
+    int W_ring;
+    DeviceCtl ctl;
 };
 cudaError_t launch_prefill_f32(const F32PrefillArgs &a, cudaStream_t s);
 

@@ -93,6 +93,19 @@ def decode_inputs(B, Hq, Hkv, d, W, dtype, seed, pos_lo, pos_hi):
     return q, kc, vc, k_new, v_new, pos
 
 
+def chunk_inputs(B, n, Hq, Hkv, d, W, dtype, seed):
+    """A chunk q [B,n,Hq,d], k/v [B,n,Hkv,d] and rings k/v [B,Hkv,W,d] whose
+    every slot is filled (slots a short sequence has not reached yet hold
+    values too, which a correct reader ignores)."""
+    g = _gen(seed)
+    q = randn((B, n, Hq, d), dtype, g)
+    k = randn((B, n, Hkv, d), dtype, g)
+    v = randn((B, n, Hkv, d), dtype, g)
+    kc = randn((B, Hkv, W, d), dtype, g)
+    vc = randn((B, Hkv, W, d), dtype, g)
+    return q, k, v, kc, vc
+
+
 def make(w: Workload):
     """Inputs of a named workload as a dict of CPU tensors."""
     if w.kind == "prefill":

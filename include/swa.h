@@ -88,6 +88,32 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
                               swa_dtype dt, void *stream);
 
 /*
+ * Causal prefill of a chunk of n new tokens that continues sequences whose
+ * earlier tokens are already in the W-slot rings: token t of batch row b is
+ * at position P = pos[b]+t and sees the keys at positions max(0,P-W+1) .. P
+ * (robocikowo.com opening definition).  Keys at positions >= pos[b] are rows
+ * of k/v; earlier ones are read from ring slot (position mod W) (Ultralytics
+ * ring-buffer paragraph), so the rings must hold positions
+ * max(0,pos[b]-W+1) .. pos[b]-1 and must not yet hold the chunk: append the
+ * chunk with swa_cache_append after this call.  The pages state no chunked
+ * form; it is the causal definition above with the keys split between the
+ * ring and the chunk, and equals rows pos[b] .. pos[b]+n-1 of swa_prefill
+ * over the whole sequence.
+ *   q, o             : [B,n,Hq,d]       k, v : [B,n,Hkv,d]
+ *   k_cache, v_cache : [B,Hkv,W,d], read only
+ *   pos              : device int32 [B], >= 0 (a negative entry is read as 0
+ *                      and records SWA_ERR_INVALID_ARG in the device status
+ *                      word)
+ *   lse              : nullable fp32 [B,Hq,n]
+ *   Other arguments as swa_prefill (bf16: d in {32, 64, 128}; fp32: d <= 128
+ *   and d % 4 == 0).
+ */
+swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *o, float *lse,
+                             const void *k_cache, const void *v_cache, const int32_t *pos,
+                             int B, int n, int Hq, int Hkv, int d, int W, float scale,
+                             swa_dtype dt, void *stream);
+
+/*
  * Ring-cache append: token t of batch row b (absolute position pos[b]+t)
  * goes to slot (pos[b]+t) mod W of that row's ring, overwriting the oldest
  * entry (Ultralytics ring-buffer paragraph; robocikowo.com rolling-buffer

@@ -84,6 +84,21 @@ def test_prefill_global_rejects(lib):
     assert f(NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, 16, 2, 2, 64, 8, 0.125, 1, NULL) == 0
 
 
+def test_prefill_chunk_rejects(lib):
+    f = lib.swa_prefill_chunk
+    call = lambda kc=FAKE, vc=FAKE, pos=FAKE, B=1, n=16, Hq=4, Hkv=2, d=64, W=32, dt=1: f(
+        FAKE, FAKE, FAKE, FAKE, NULL, kc, vc, pos, B, n, Hq, Hkv, d, W, 0.125, dt, NULL)
+    assert call(pos=NULL) == 1
+    assert call(kc=NULL) == 1
+    assert call(vc=MISALIGNED) == 1
+    assert call(pos=ctypes.c_void_p((1 << 20) + 2)) == 1   # int32 positions need 4-byte alignment
+    assert call(W=0) == 1
+    assert call(d=48) == 2
+    assert call(Hq=3) == 1
+    assert call(n=0, kc=NULL, vc=NULL, pos=NULL) == 0
+    assert call(B=0, kc=NULL, vc=NULL, pos=NULL) == 0
+
+
 def test_append_rejects(lib):
     f = lib.swa_cache_append
     assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1      # no pos
