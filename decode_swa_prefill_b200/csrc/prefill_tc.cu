@@ -52,6 +52,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "swa_internal.h"
 
@@ -169,7 +171,8 @@ __device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
     return q.active ? (q.te - q.ts) + n_glob : 0;
 }
 
-__device__ __forceinline__ Work make_work(const TcPrefillArgs &a, int n_mode1)
+template <bool RING>
+__device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, int n_mode1)
 {
     Work w;
     const int G = a.Hq / a.Hkv;
@@ -220,27 +223,49 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, int n_mode1)
                 if (qt < nqt) w.q[x] = QTile{h, qt * BM, 0, min(BM, a.T - qt * BM), 0, 0, true};
             }
         }
-        // a chunk continuing a ring starts at position pos[b] (a negative
-        // entry is read as 0; the producer records it)
-        const long long p0 = a.pos ? max((long long)a.pos[w.b], 0LL) : 0LL;
-        w.p0 = p0;
-        w.kend = p0 + a.T;
-        long long lo = w.kend, hi = -1;
-        long long lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
-        for (int x = 0; x < 2; ++x) {
-            if (!w.q[x].active) continue;
-            lo_x[x] = max(0LL, p0 + w.q[x].m0 - a.left);
-            hi_x[x] = min(w.kend - 1, p0 + w.q[x].m0 + BM - 1 + a.right);
-            lo = min(lo, lo_x[x]);
-            hi = max(hi, hi_x[x]);
-        }
-        w.j_lo = (int)(lo / BN);
-        w.n_band = (int)(hi / BN) - w.j_lo + 1;
-        for (int x = 0; x < 2; ++x)
-            if (w.q[x].active) {
-                w.q[x].ts = (int)(lo_x[x] / BN) - w.j_lo;
-                w.q[x].te = (int)(hi_x[x] / BN) - w.j_lo + 1;
+        if constexpr (RING) {
+            // a chunk continuing a ring starts at position pos[b] (a
+            // negative entry is read as 0; the producer records it); key
+            // tiles are counted in absolute positions
+            const long long p0 = max((long long)ring.pos[w.b], 0LL);
+            w.p0 = p0;
+            w.kend = p0 + a.T;
+            long long lo = w.kend, hi = -1;
+            long long lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+            for (int x = 0; x < 2; ++x) {
+                if (!w.q[x].active) continue;
+                lo_x[x] = max(0LL, p0 + w.q[x].m0 - a.left);
+                hi_x[x] = min(w.kend - 1, p0 + w.q[x].m0 + BM - 1 + a.right);
+                lo = min(lo, lo_x[x]);
+                hi = max(hi, hi_x[x]);
             }
+            w.j_lo = (int)(lo / BN);
+            w.n_band = (int)(hi / BN) - w.j_lo + 1;
+            for (int x = 0; x < 2; ++x)
+                if (w.q[x].active) {
+                    w.q[x].ts = (int)(lo_x[x] / BN) - w.j_lo;
+                    w.q[x].te = (int)(hi_x[x] / BN) - w.j_lo + 1;
+                }
+        } else {
+            w.p0 = 0;
+            w.kend = a.T;
+            int lo = a.T, hi = -1;
+            int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+            for (int x = 0; x < 2; ++x) {
+                if (!w.q[x].active) continue;
+                lo_x[x] = max(0, w.q[x].m0 - a.left);
+                hi_x[x] = min(a.T - 1, w.q[x].m0 + BM - 1 + a.right);
+                lo = min(lo, lo_x[x]);
+                hi = max(hi, hi_x[x]);
+            }
+            w.j_lo = lo / BN;
+            w.n_band = hi / BN - w.j_lo + 1;
+            for (int x = 0; x < 2; ++x)
+                if (w.q[x].active) {
+                    w.q[x].ts = lo_x[x] / BN - w.j_lo;
+                    w.q[x].te = hi_x[x] / BN - w.j_lo + 1;
+                }
+        }
         w.n_glob = (a.gidx != nullptr && a.g > 0) ? (a.g + BN - 1) / BN : 0;
     }
     w.hk = w.q[0].h / G;
@@ -391,12 +416,14 @@ __device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillAr
     l += tot.x + tot.y;
 }
 
-template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                          const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
-                          const TcPrefillArgs a, const int n_mode1)
+// The whole CTA program.  RING: a chunk continuing a ring
+// (swa_prefill_chunk), compiled as its own kernel so that the other calls
+// keep 32-bit key positions, no ring branches and their four-map argument
+// list (two more tensor-map arguments alone cost those launches 2%).
+template <int D, bool RING>
+__device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                                            const CUtensorMap *tmO, const CUtensorMap *tmKr, const CUtensorMap *tmVr,
+                                            const TcPrefillArgs &a, const RingArgs &ring, const int n_mode1)
 {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -408,7 +435,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const Work w = make_work(a, n_mode1);
+    const Work w = make_work<RING>(a, ring, n_mode1);
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -433,10 +460,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_mbar_init();
     }
     if (warp == 8 && lane == 0) {
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-        prefetch_tensormap(&tmO);
+        prefetch_tensormap(tmQ);
+        prefetch_tensormap(tmK);
+        prefetch_tensormap(tmV);
+        prefetch_tensormap(tmO);
     }
     if (warp == 9) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tc_fence_before();
@@ -458,7 +485,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int x = 0; x < 2; ++x)
                     if (w.q[x].active)
                         for (int ch = 0; ch < C::NCH; ++ch)
-                            tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, &tmQ, &bars->q_full, ch * C::E, w.q[x].h,
+                            tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, tmQ, &bars->q_full, ch * C::E, w.q[x].h,
                                         w.q[x].m0, w.b);
             }
         } else {
@@ -470,61 +497,108 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->q_full);
         }
-        if (a.pos && lane == 0 && a.pos[w.b] < 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
-        // One K or V key tile into stage st: a TMA tile of the key tensor or
-        // of the ring, or 16-byte cp.async row copies (global keys; ring rows
-        // that wrap around the ring's end or meet the chunk's first row).
-        auto load_tile = [&](bool is_v, int st, int t) {
-            uint8_t *dst = (is_v ? sV : sK) + st * C::KTILE;
-            uint64_t *bar = is_v ? &bars->v_full[st] : &bars->k_full[st];
-            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(is_v ? a.v : a.k);
-            if (t >= w.n_band) {
-                const int gt = t - w.n_band;
-                gather_tile<D>(dst, BN, C::KCH, src, gb + gt * BN, min(BN, a.g - gt * BN), w.b, a.T, a.Hkv, w.hk,
-                               lane);
-            } else {
-                const long long key0 = (long long)(w.j_lo + t) * BN;
-                const bool ring_tile = a.pos && key0 < w.p0;
-                const long long slot0 = ring_tile ? key0 % a.W_ring : 0;
-                if (!ring_tile || (key0 + BN <= w.p0 && slot0 + BN <= a.W_ring)) {
-                    if (lane == 0) {
-                        mbar_expect_tx(bar, C::KTILE);
-                        for (int ch = 0; ch < C::NCH; ++ch) {
-                            if (ring_tile)
-                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmVr : &tmKr, bar, ch * C::E, (int)slot0, w.hk,
-                                            w.b);
-                            else
-                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk,
-                                            (int)(key0 - w.p0), w.b);
+        if (RING && lane == 0 && ring.pos[w.b] < 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+        if constexpr (RING) {
+            const long long p0 = RING ? w.p0 : 0;
+            // One K or V key tile into stage st: a TMA tile of the key tensor or
+            // of the ring, or 16-byte cp.async row copies (global keys; ring rows
+            // that wrap around the ring's end or meet the chunk's first row).
+            auto load_tile = [&](bool is_v, int st, int t) {
+                uint8_t *dst = (is_v ? sV : sK) + st * C::KTILE;
+                uint64_t *bar = is_v ? &bars->v_full[st] : &bars->k_full[st];
+                const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(is_v ? a.v : a.k);
+                if (t >= w.n_band) {
+                    const int gt = t - w.n_band;
+                    gather_tile<D>(dst, BN, C::KCH, src, gb + gt * BN, min(BN, a.g - gt * BN), w.b, a.T, a.Hkv, w.hk,
+                                   lane);
+                } else {
+                    const long long key0 = (long long)(w.j_lo + t) * BN;
+                    const bool ring_tile = RING && key0 < w.p0;
+                    const long long slot0 = ring_tile ? key0 % ring.W : 0;
+                    if (!RING || !ring_tile || (key0 + BN <= w.p0 && slot0 + BN <= ring.W)) {
+                        if (lane == 0) {
+                            mbar_expect_tx(bar, C::KTILE);
+                            for (int ch = 0; ch < C::NCH; ++ch) {
+                                if (ring_tile)
+                                    tma_load_4d(dst + ch * C::KCH, is_v ? tmVr : tmKr, bar, ch * C::E, (int)slot0, w.hk,
+                                                w.b);
+                                else
+                                    tma_load_4d(dst + ch * C::KCH, is_v ? tmV : tmK, bar, ch * C::E, w.hk,
+                                                (int)(key0 - p0), w.b);
+                            }
                         }
+                        return;
                     }
-                    return;
+                    if (!RING) return;
+                    const __nv_bfloat16 *rc = static_cast<const __nv_bfloat16 *>(is_v ? ring.vc : ring.kc);
+                    gather_rows<D>(dst, BN, C::KCH, src, lane, [&](int r) -> const __nv_bfloat16 * {
+                        const long long p = key0 + r;
+                        if (p >= p0) {
+                            const long long row = p - p0;
+                            return row < a.T ? src + (((long long)w.b * a.T + row) * a.Hkv + w.hk) * D : nullptr;
+                        }
+                        return rc + (((long long)w.b * a.Hkv + w.hk) * ring.W + p % ring.W) * D;
+                    });
                 }
-                const __nv_bfloat16 *ring = static_cast<const __nv_bfloat16 *>(is_v ? a.vc : a.kc);
-                gather_rows<D>(dst, BN, C::KCH, src, lane, [&](int r) -> const __nv_bfloat16 * {
-                    const long long p = key0 + r;
-                    if (p >= w.p0) {
-                        const long long row = p - w.p0;
-                        return row < a.T ? src + (((long long)w.b * a.T + row) * a.Hkv + w.hk) * D : nullptr;
-                    }
-                    return ring + (((long long)w.b * a.Hkv + w.hk) * a.W_ring + p % a.W_ring) * D;
-                });
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar);
+            };
+            for (int t = 0; t < w.n_tiles && ok; ++t) {
+                const int st = t % NSTAGE;
+                const uint32_t par = ((t / NSTAGE) & 1) ^ 1;
+                ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
+                if (!ok) break;
+                load_tile(false, st, t);
+                kiss[st]++;
+                ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
+                if (!ok) break;
+                load_tile(true, st, t);
+                viss[st]++;
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar);
-        };
-        for (int t = 0; t < w.n_tiles && ok; ++t) {
-            const int st = t % NSTAGE;
-            const uint32_t par = ((t / NSTAGE) & 1) ^ 1;
-            ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
-            if (!ok) break;
-            load_tile(false, st, t);
-            kiss[st]++;
-            ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
-            if (!ok) break;
-            load_tile(true, st, t);
-            viss[st]++;
+        } else {
+            for (int t = 0; t < w.n_tiles && ok; ++t) {
+                const bool band = t < w.n_band;
+                const int key0 = (w.j_lo + t) * BN;
+                const int gt = t - w.n_band;
+                const int nr = band ? 0 : min(BN, a.g - gt * BN);
+                const int st = t % NSTAGE;
+                const uint32_t par = ((t / NSTAGE) & 1) ^ 1;
+                ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
+                if (!ok) break;
+                if (band) {
+                    if (lane == 0) {
+                        mbar_expect_tx(&bars->k_full[st], C::KTILE);
+                        for (int ch = 0; ch < C::NCH; ++ch)
+                            tma_load_4d(sK + st * C::KTILE + ch * C::KCH, tmK, &bars->k_full[st], ch * C::E, w.hk,
+                                        key0, w.b);
+                    }
+                } else {
+                    gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
+                                   gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->k_full[st]);
+                }
+                kiss[st]++;
+                ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
+                if (!ok) break;
+                if (band) {
+                    if (lane == 0) {
+                        mbar_expect_tx(&bars->v_full[st], C::KTILE);
+                        for (int ch = 0; ch < C::NCH; ++ch)
+                            tma_load_4d(sV + st * C::KTILE + ch * C::KCH, tmV, &bars->v_full[st], ch * C::E, w.hk,
+                                        key0, w.b);
+                    }
+                } else {
+                    gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
+                                   gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->v_full[st]);
+                }
+                viss[st]++;
+            }
         }
         if (!ok && lane == 0) {
             // let our own copies land before the CTA's shared memory goes away
@@ -626,13 +700,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const QTile qt = x ? w.q[1] : w.q[0];
         const int n_band = w.n_band;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        // key positions: 64-bit only for a chunk continuing a ring
+        typedef typename std::conditional<RING, long long, int>::type kpos_t;
+        const long long p0 = RING ? w.p0 : 0;
+#define KEND (RING ? (kpos_t)w.kend : (kpos_t)a.T) // one past the last key
         long long i_row;                        // absolute query position
-        if (w.mode == 0) i_row = w.p0 + qt.m0 + r;
+        if (w.mode == 0) i_row = p0 + qt.m0 + r;
         else i_row = (qt.active && r < qt.nrows) ? gb[qt.gt * BM + r] : 0;
-        const long long i_out = i_row - w.p0;   // row in q / o / lse
+        const long long i_out = i_row - p0;     // row in q / o / lse
         const bool row_real = qt.active && r < qt.nrows;
         const bool warp_has_rows = qt.active && quarter * 32 < qt.nrows;
-        const long long wi0 = w.p0 + qt.m0 + quarter * 32, wi1 = wi0 + 31;
+        const long long wi0 = p0 + qt.m0 + quarter * 32, wi1 = wi0 + 31;
         float m = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         for (int t = 0; t < w.n_tiles && qt.active; ++t) {
@@ -644,21 +722,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
             // ---- which 32-key chunks can any row of this warp see ----
             const bool band = t < w.n_band;
-            const long long key0 = (long long)(w.j_lo + t) * BN;
+            const kpos_t key0 = (kpos_t)(w.j_lo + t) * BN;
             int c_lo = 0, c_hi = -1;
             bool interior = false;
             if (warp_has_rows) {
                 if (w.mode == 1) {
-                    c_hi = (int)((min(key0 + BN - 1, w.kend - 1) - key0) / 32);
-                    interior = key0 + BN <= w.kend;
+                    c_hi = (int)((min(key0 + BN - 1, KEND - 1) - key0) / 32);
+                    interior = key0 + BN <= KEND;
                 } else if (band) {
-                    const long long lo = max(max(key0, wi0 - a.left), 0LL);
-                    const long long hi = min(min(key0 + BN - 1, wi1 + a.right), w.kend - 1);
+                    const long long lo = max(max((long long)key0, wi0 - a.left), 0LL);
+                    const long long hi = min(min((long long)key0 + BN - 1, wi1 + a.right), (long long)KEND - 1);
                     if (lo <= hi) {
                         c_lo = (int)((lo - key0) / 32);
                         c_hi = (int)((hi - key0) / 32);
                     }
-                    interior = (key0 + BN - 1 < w.kend) && band_contains(wi1, key0, a.left, a.right) &&
+                    interior = (key0 + BN - 1 < KEND) && band_contains(wi1, key0, a.left, a.right) &&
                                band_contains(wi0, key0 + BN - 1, a.left, a.right);
                 } else {
                     c_hi = (min(BN, a.g - (t - w.n_band) * BN) - 1) / 32;
@@ -673,10 +751,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             k.col_hi = BN - 1;
             k.by_range = (w.mode == 1) || band;
             if (w.mode == 1) {
-                k.col_hi = (int)min((long long)BN - 1, w.kend - 1 - key0);
+                k.col_hi = (int)min((kpos_t)BN - 1, KEND - 1 - key0);
             } else if (band) {
                 k.col_lo = (int)max(i_row - a.left - key0, 0LL);
-                k.col_hi = (int)min(min(i_row + a.right, w.kend - 1) - key0, (long long)BN - 1);
+                k.col_hi = (int)min(min(i_row + a.right, (long long)KEND - 1) - key0, (long long)BN - 1);
             }
             k.gc_base = (t - w.n_band) * BN;
             k.i_row = i_row;
@@ -770,7 +848,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0) mbar_arrive(&bars->epi[x]);
             if (r == 0 && wait_bounded(&bars->epi[x], 0, ctl) && !bars->abort) {
                 for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_store_4d(&tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
+                    tma_store_4d(tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
                 tma_store_commit();
                 tma_store_wait_all();
             }
@@ -783,6 +861,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                          const TcPrefillArgs a, const int n_mode1)
+{
+    prefill_cta<D, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    swa_prefill_ring_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                            const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
+                            const TcPrefillArgs a, const RingArgs ring, const int n_mode1)
+{
+    prefill_cta<D, true>(&tmQ, &tmK, &tmV, &tmO, &tmKr, &tmVr, a, ring, n_mode1);
 }
 
 // ------------------------------------------------------------------ host --
@@ -842,16 +939,16 @@ bool make_ring_map(CUtensorMap *m, const void *ptr, int B, int Hkv, int W)
     return r == CUDA_SUCCESS;
 }
 
-template <int D>
-cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
+template <int D, bool RING>
+cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     using C = Cfg<D>;
     CUtensorMap mq, mk, mv, mo, mkr, mvr;
     if (!make_map<D>(&mq, a.q, a.B, a.T, a.Hq, BM) || !make_map<D>(&mk, a.k, a.B, a.T, a.Hkv, BN) ||
         !make_map<D>(&mv, a.v, a.B, a.T, a.Hkv, BN) || !make_map<D>(&mo, a.o, a.B, a.T, a.Hq, BM))
         return cudaErrorInvalidValue;
-    if (a.pos) {
-        if (!make_ring_map<D>(&mkr, a.kc, a.B, a.Hkv, a.W_ring) || !make_ring_map<D>(&mvr, a.vc, a.B, a.Hkv, a.W_ring))
+    if (RING) {
+        if (!make_ring_map<D>(&mkr, ring.kc, a.B, a.Hkv, ring.W) || !make_ring_map<D>(&mvr, ring.vc, a.B, a.Hkv, ring.W))
             return cudaErrorInvalidValue;
     } else {
         mkr = mk; // unused without a ring
@@ -861,8 +958,10 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(swa_prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
+        cudaError_t e = RING ? cudaFuncSetAttribute(swa_prefill_ring_kernel<D>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                             : cudaFuncSetAttribute(swa_prefill_tc_kernel<D>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -884,20 +983,29 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, cudaStream_t s)
     }
     const int grid = n_mode0 + n_mode1;
     if (grid == 0) return cudaSuccess;
-    swa_prefill_tc_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, n_mode1);
+    if (RING)
+        swa_prefill_ring_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring, n_mode1);
+    else
+        swa_prefill_tc_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, n_mode1);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
+{
+    return ring.pos ? launch_dr<D, true>(mode, a, ring, s) : launch_dr<D, false>(mode, a, ring, s);
 }
 
 }  // namespace
 
 // mode 0: band tiles (+ dense global-row CTAs first in the same grid when
 // global tokens are present); mode 1: dense global rows only.
-cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, cudaStream_t s)
+cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     switch (d) {
-    case 32: return launch_d<32>(mode, a, s);
-    case 64: return launch_d<64>(mode, a, s);
-    case 128: return launch_d<128>(mode, a, s);
+    case 32: return launch_d<32>(mode, a, ring, s);
+    case 64: return launch_d<64>(mode, a, ring, s);
+    case 128: return launch_d<128>(mode, a, ring, s);
     default: return cudaErrorInvalidValue;
     }
 }

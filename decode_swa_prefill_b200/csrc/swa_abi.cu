@@ -111,7 +111,7 @@ swa_status swa_prefill(const void *q, const void *k, const void *v, void *o, flo
     a.lse = lse; a.gidx = nullptr; a.g = 0;
     a.q = q; a.k = k; a.v = v; a.o = o;
     if ((st = ctl(&a.ctl)) != SWA_OK) return st;
-    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
 }
 
 swa_status swa_prefill_global(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -138,7 +138,7 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
     a.lse = lse; a.gidx = g > 0 ? global_idx : nullptr; a.g = g;
     a.q = q; a.k = k; a.v = v; a.o = o;
     if ((st = ctl(&a.ctl)) != SWA_OK) return st;
-    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
 }
 
 swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *o, float *lse, const void *k_cache,
@@ -167,9 +167,8 @@ swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *
     a.scale_log2 = scale * 1.4426950408889634f;
     a.lse = lse; a.gidx = nullptr; a.g = 0;
     a.q = q; a.k = k; a.v = v; a.o = o;
-    a.pos = pos; a.kc = k_cache; a.vc = v_cache; a.W_ring = W;
     if ((st = ctl(&a.ctl)) != SWA_OK) return st;
-    return from_cuda(swa::launch_prefill_tc(d, 0, a, s));
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{pos, k_cache, v_cache, W}, s));
 }
 
 swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new, const int32_t *pos,

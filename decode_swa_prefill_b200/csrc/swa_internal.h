@@ -34,19 +34,23 @@ struct TcPrefillArgs {
     int g;
     const void *q, *k, *v;    // raw pointers (gathers)
     void *o;                  // raw output pointer (scatter in global-row mode)
-    // chunk continuing a ring (band mode): T is the chunk length n, query row
-    // r of batch b is at position pos[b]+r; keys before pos[b] come from the
-    // W_ring-slot caches kc / vc [B,Hkv,W_ring,d]
+    DeviceCtl ctl;
+};
+
+// A chunk continuing a ring (band mode): T is the chunk length n, query row r
+// of batch b is at position pos[b]+r, and keys before pos[b] come from the
+// W-slot caches kc / vc [B,Hkv,W,d].  A separate kernel argument, so that the
+// other launches keep their argument layout.
+struct RingArgs {
     const int32_t *pos;       // null: no ring
     const void *kc, *vc;
-    int W_ring;
-    DeviceCtl ctl;
+    int W;
 };
 
 // mode 0: one CTA per (q tile, head, batch) over band tiles (+ one gathered
 //         tile of global keys per 128 globals when gidx != null)
 // mode 1: one CTA per (128 global rows, head, batch): dense rows over all keys
-cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s);
 
 // ---- SIMT kernels ----
 struct F32PrefillArgs {

@@ -19,9 +19,9 @@ import torch
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # "prefill" | "prefill_global" | "decode"
+    kind: str              # "prefill" | "prefill_global" | "decode" | "prefill_chunk"
     B: int
-    T: int                 # sequence length (prefill) or ring size W (decode)
+    T: int                 # sequence length (prefill), ring size W (decode), chunk length (chunk)
     Hq: int
     Hkv: int
     d: int
@@ -29,7 +29,7 @@ class Workload:
     dtype: torch.dtype
     seed: int
     g: int = 0             # global tokens per sequence (prefill_global)
-    pos_lo: int = 0        # decode: current positions drawn from [pos_lo, pos_hi)
+    pos_lo: int = 0        # decode / chunk: positions drawn from [pos_lo, pos_hi)
     pos_hi: int = 0
     notes: str = field(default="", compare=False)
 
@@ -50,7 +50,13 @@ MISTRAL_DECODE = Workload("mistral7b_decode_B64_h32x8_d128_W4096", "decode", B=6
 LONGFORMER = Workload("longformer_prefill_B8_T4096_h12_d64_W512_g16", "prefill_global", B=8,
                       T=4096, Hq=12, Hkv=12, d=64, W=512, dtype=torch.bfloat16, seed=4, g=16)
 
-ALL = [TOY, TINYMISTRAL, MISTRAL_PREFILL, MISTRAL_DECODE, LONGFORMER]
+# serving-path continuation: a 4096-token chunk of each of 4 sequences whose
+# earlier tokens are in full W=4096 rings (Mistral-7B shapes)
+MISTRAL_CHUNK = Workload("mistral7b_chunk_B4_n4096_h32x8_d128_W4096", "prefill_chunk", B=4, T=4096,
+                         Hq=32, Hkv=8, d=128, W=4096, dtype=torch.bfloat16, seed=5,
+                         pos_lo=4096, pos_hi=131072)
+
+ALL = [TOY, TINYMISTRAL, MISTRAL_PREFILL, MISTRAL_DECODE, LONGFORMER, MISTRAL_CHUNK]
 
 
 def _gen(seed: int) -> torch.Generator:
@@ -118,4 +124,9 @@ def make(w: Workload):
         q, kc, vc, kn, vn, pos = decode_inputs(w.B, w.Hq, w.Hkv, w.d, w.W, w.dtype, w.seed,
                                                w.pos_lo, w.pos_hi)
         return {"q": q, "k_cache": kc, "v_cache": vc, "k_new": kn, "v_new": vn, "pos": pos}
+    if w.kind == "prefill_chunk":
+        q, k, v, kc, vc = chunk_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.W, w.dtype, w.seed)
+        pos = torch.randint(w.pos_lo, w.pos_hi, (w.B,), generator=_gen(w.seed + 2000),
+                            dtype=torch.int64).to(torch.int32)
+        return {"q": q, "k": k, "v": v, "k_cache": kc, "v_cache": vc, "pos": pos}
     raise ValueError(w.kind)

@@ -25,6 +25,13 @@ def test_global_pairs_match_oracle(T, W, g):
     assert bench.global_pairs(T, W, gi) == oracle.count_pairs(T, W, oracle.SYMMETRIC, gi if g else None)
 
 
+@pytest.mark.parametrize("n,W,p0", [(10, 4, 0), (10, 4, 2), (5, 100, 3), (7, 3, 50), (1, 1, 0), (300, 256, 0),
+                                     (4096, 4096, 5000)])
+def test_chunk_pairs_match_oracle(n, W, p0):
+    # rows p0..p0+n-1 of a causal prefill over p0+n tokens
+    assert bench.chunk_pairs(n, W, p0) == oracle.count_pairs(p0 + n, W) - oracle.count_pairs(p0, W)
+
+
 def test_step_accounting_totals():
     acc = bench.step_accounting(wl.make(wl.LONGFORMER))
     assert acc["f_prefill"] == 125_831_168 * 32 * 4 * 128
