@@ -54,6 +54,16 @@ def _load():
         lib.oracle_swa_prefill_chunk.argtypes = [p, p, p, p, p, p, p, p, c_long, c_long, c_long, c_long,
                                                  c_long, c_long, c_double]
         lib.oracle_swa_prefill_chunk.restype = c_int
+        lib.oracle_sink_allowed.argtypes = [c_long, c_long, c_long, c_long, c_long]
+        lib.oracle_sink_allowed.restype = c_int
+        lib.oracle_count_pairs_sinks.argtypes = [c_long, c_long, c_long]
+        lib.oracle_count_pairs_sinks.restype = ctypes.c_longlong
+        lib.oracle_swa_prefill_sinks.argtypes = [p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
+                                                 c_long, c_long, c_double, p, c_long, c_int]
+        lib.oracle_swa_prefill_sinks.restype = c_int
+        lib.oracle_swa_decode_sinks.argtypes = [p, p, p, p, p, p, p, p, c_long, c_long, c_long, c_long,
+                                                c_long, c_long, c_double]
+        lib.oracle_swa_decode_sinks.restype = c_int
         _lib = lib
     return _lib
 
@@ -218,6 +228,50 @@ def swa_prefill_chunk(q, k, v, k_cache, v_cache, pos, scale=None):
     o = np.zeros((B, n, Hq, d)); lse = np.zeros((B, Hq, n))
     rc = _load().oracle_swa_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc), _ptr(_i32(pos)),
                                           _ptr(o), _ptr(lse), B, n, Hq, Hkv, d, W, float(scale))
+    if rc != 0:
+        raise ValueError("negative position")
+    return o, lse
+
+
+# ------------------------------------------------------------------ sinks --
+
+def sink_allowed(i, j, T, W, s):
+    """Causal window plus the first s tokens as attention sinks (Ultralytics
+    glossary, related-terms entry on attention sinks)."""
+    return bool(_load().oracle_sink_allowed(i, j, T, W, s))
+
+
+def count_pairs_sinks(T, W, s):
+    return int(_load().oracle_count_pairs_sinks(T, W, s))
+
+
+def swa_prefill_sinks(q, k, v, W, sinks, scale=None, rows=None, nthreads=None):
+    """Causal window W plus the first `sinks` tokens of each sequence; shapes
+    and row selection as swa_prefill."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = _rows_arg(rows, B, Hq, T)
+    o = np.zeros((len(r), d)); lse = np.zeros(len(r))
+    _load().oracle_swa_prefill_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
+                                     int(sinks), float(scale), _ptr(r), len(r), nthreads or default_threads())
+    return _unflatten(o, lse, r, rows is None, B, T, Hq, d)
+
+
+def swa_decode_sinks(q, k_cache, v_cache, k_sink, v_sink, pos, scale=None):
+    """One decode step over the ring plus sink caches [B,Hkv,s,d] holding
+    positions 0..s-1 (the current token already appended to the ring)."""
+    q, kc, vc, ks, vs = _f64(q), _f64(k_cache), _f64(v_cache), _f64(k_sink), _f64(v_sink)
+    B, Hq, d = q.shape
+    Hkv, W = kc.shape[1], kc.shape[2]
+    s = ks.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, Hq, d)); lse = np.zeros((B, Hq))
+    rc = _load().oracle_swa_decode_sinks(_ptr(q), _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(_i32(pos)),
+                                         _ptr(o), _ptr(lse), B, Hq, Hkv, d, W, s, float(scale))
     if rc != 0:
         raise ValueError("negative position")
     return o, lse

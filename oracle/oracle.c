@@ -37,6 +37,7 @@
 
 #define ORACLE_CAUSAL 0
 #define ORACLE_SYMMETRIC 1
+#define ORACLE_SINKS 2
 
 /* ---------------------------------------------------------------- masks -- */
 
@@ -67,6 +68,25 @@ int oracle_allowed(long i, long j, long T, long W, int mode, const int32_t *gidx
     if (j < 0 || j >= T || i < 0 || i >= T) return 0;
     if (g > 0 && (is_global(i, gidx, g) || is_global(j, gidx, g))) return 1;
     return oracle_in_window(i, j, T, W, mode);
+}
+
+/* Causal window plus attention sinks [P4 related-terms entry on attention
+ * sinks: StreamingLLM keeps the first tokens of a sequence in the cache
+ * beside the window]: query i sees key j <= i when j lies in the window
+ * (j >= i-W+1) or is one of the first s tokens (j < s). */
+int oracle_sink_allowed(long i, long j, long T, long W, long s)
+{
+    if (j < 0 || j >= T || i < 0 || i >= T || j > i) return 0;
+    return j >= i - W + 1 || j < s;
+}
+
+/* Pairs a causal window with s sinks allows. */
+long long oracle_count_pairs_sinks(long T, long W, long s)
+{
+    long long n = 0;
+    for (long i = 0; i < T; i++)
+        for (long j = 0; j < T; j++) n += oracle_sink_allowed(i, j, T, W, s);
+    return n;
 }
 
 /* The explicit [T,T] boolean mask (the brute-force form the pages warn
@@ -181,6 +201,7 @@ typedef struct {
     int mode;
     const int32_t *gidx; /* [B,g] or NULL */
     long g;
+    long sinks;          /* causal window plus the first `sinks` tokens (mode ORACLE_SINKS) */
     double scale;
     const int64_t *rows; /* flattened (b*Hq + h)*T + i */
     long nrows;
@@ -198,7 +219,9 @@ static void prefill_one(prefill_job *J, long r, const double **kr, const double 
     const int32_t *gb = J->gidx ? J->gidx + b * J->g : NULL;
     long n = 0;
     for (long j = 0; j < J->T; j++) {
-        if (!oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0)) continue;
+        const int ok = J->mode == ORACLE_SINKS ? oracle_sink_allowed(i, j, J->T, J->W, J->sinks)
+                                               : oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0);
+        if (!ok) continue;
         kr[n] = J->k + ((b * J->T + j) * J->Hkv + hk) * J->d;
         vr[n] = J->v + ((b * J->T + j) * J->Hkv + hk) * J->d;
         n++;
@@ -248,7 +271,7 @@ int oracle_swa_prefill(const double *q, const double *k, const double *v, double
                        long B, long T, long Hq, long Hkv, long d, long W, double scale,
                        const int64_t *rows, long nrows, int nthreads)
 {
-    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_CAUSAL, NULL, 0, scale, rows, nrows};
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_CAUSAL, NULL, 0, 0, scale, rows, nrows};
     return run_prefill(&J, nthreads);
 }
 
@@ -260,7 +283,17 @@ int oracle_swa_prefill_global(const double *q, const double *k, const double *v,
                               long B, long T, long Hq, long Hkv, long d, long W, double scale,
                               const int64_t *rows, long nrows, int nthreads)
 {
-    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SYMMETRIC, g > 0 ? gidx : NULL, g, scale, rows, nrows};
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SYMMETRIC, g > 0 ? gidx : NULL, g, 0, scale, rows, nrows};
+    return run_prefill(&J, nthreads);
+}
+
+/* Causal window plus the first s tokens as attention sinks [P4 related-terms
+ * entry on attention sinks; P3 opening definition for the window]. */
+int oracle_swa_prefill_sinks(const double *q, const double *k, const double *v, double *o, double *lse,
+                             long B, long T, long Hq, long Hkv, long d, long W, long s, double scale,
+                             const int64_t *rows, long nrows, int nthreads)
+{
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SINKS, NULL, 0, s, scale, rows, nrows};
     return run_prefill(&J, nthreads);
 }
 
@@ -343,5 +376,46 @@ int oracle_swa_prefill_chunk(const double *q, const double *k, const double *v, 
         }
     }
     free(kr); free(vr); free(s);
+    return 0;
+}
+
+/* One decode step with attention sinks beside the ring [P4 related-terms
+ * entry: StreamingLLM keeps the first tokens in the cache beside the window;
+ * P4 ring-buffer paragraph].  The token at position P = pos[b] is already in
+ * the ring, whose filled slots 0..min(P+1,W)-1 hold the window; the sink
+ * caches [B,Hkv,s,d] hold positions 0..s-1, of which those older than the
+ * window (position < P-W+1) are added; the others are still in the ring and
+ * count once.  Keys in list order: sinks, then ring slots. */
+int oracle_swa_decode_sinks(const double *q, const double *kc, const double *vc, const double *ks,
+                            const double *vs, const int32_t *pos, double *o, double *lse, long B, long Hq,
+                            long Hkv, long d, long W, long s, double scale)
+{
+    for (long b = 0; b < B; b++)
+        if (pos[b] < 0) return -1;
+    const double **kr = malloc(sizeof(double *) * (size_t)(W + s));
+    const double **vr = malloc(sizeof(double *) * (size_t)(W + s));
+    double *sc = malloc(sizeof(double) * (size_t)(W + s));
+    for (long b = 0; b < B; b++) {
+        const long P = pos[b];
+        const long nvalid = P + 1 < W ? P + 1 : W;
+        long nsink = P - W + 1 < s ? P - W + 1 : s;
+        if (nsink < 0) nsink = 0;
+        for (long h = 0; h < Hq; h++) {
+            const long hk = h * Hkv / Hq;
+            long n = 0;
+            for (long j = 0; j < nsink; j++, n++) {
+                kr[n] = ks + ((b * Hkv + hk) * s + j) * d;
+                vr[n] = vs + ((b * Hkv + hk) * s + j) * d;
+            }
+            for (long sl = 0; sl < nvalid; sl++, n++) {
+                kr[n] = kc + ((b * Hkv + hk) * W + sl) * d;
+                vr[n] = vc + ((b * Hkv + hk) * W + sl) * d;
+            }
+            double l;
+            attend_row(q + (b * Hq + h) * d, kr, vr, n, d, scale, o + (b * Hq + h) * d, &l, sc);
+            if (lse) lse[b * Hq + h] = l;
+        }
+    }
+    free(kr); free(vr); free(sc);
     return 0;
 }
