@@ -16,8 +16,8 @@ import torch
 
 __all__ = [
     "SwaError", "load", "library_path", "EXPORTED",
-    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode",
-    "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
+    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_cache_append",
+    "swa_decode", "swa_decode_sinks", "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
     "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
 
@@ -29,7 +29,8 @@ SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 
 # every symbol include/swa.h declares
 EXPORTED = [
-    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode_workspace_bytes",
+    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
+    "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
     "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
@@ -56,6 +57,8 @@ def load():
     lib.swa_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.swa_prefill_global.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
     lib.swa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.swa_prefill_sinks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_decode_sinks.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -68,7 +71,8 @@ def load():
     lib.swa_set_wait_limit_ns.restype = None
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
-    for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_cache_append", "swa_decode",
+    for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
+                 "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -125,6 +129,22 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
     st = load().swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
                             float(scale), _dtype_code(q), _stream(stream))
     _check(st, "swa_prefill")
+    return o
+
+
+def swa_prefill_sinks(q, k, v, W, n_sink, scale=None, o=None, lse=None, stream=None):
+    """Causal window W plus the first n_sink tokens of each sequence as
+    attention sinks; returns o (and fills lse when given)."""
+    _dev_contig(q, k, v, o, lse)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, T, Hkv, d) and v.shape == k.shape, "k/v shape")
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(n_sink), B, T, Hq, Hkv, d, W,
+                                  float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_prefill_sinks")
     return o
 
 
@@ -200,6 +220,30 @@ def swa_decode(q, k_cache, v_cache, pos, scale=None, o=None, lse=None, workspace
                            B, Hq, Hkv, d, W, float(scale), _dtype_code(q), _ptr(workspace),
                            ws_bytes, _stream(stream))
     _check(st, "swa_decode")
+    return o
+
+
+def swa_decode_sinks(q, k_cache, v_cache, k_sink, v_sink, pos, scale=None, o=None, lse=None, workspace=None,
+                     stream=None):
+    """swa_decode plus attention sinks: k_sink/v_sink [B,Hkv,n_sink,d] hold
+    positions 0..n_sink-1 and are seen beside the window."""
+    _dev_contig(q, k_cache, v_cache, k_sink, v_sink, pos, o, lse, workspace)
+    B, Hq, d = q.shape
+    Hkv, W = k_cache.shape[1], k_cache.shape[2]
+    n_sink = k_sink.shape[2]
+    _need(k_sink.shape == (B, Hkv, n_sink, d) and v_sink.shape == k_sink.shape, "sink cache shape")
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    if o is None:
+        o = torch.empty_like(q)
+    need = swa_decode_workspace_bytes(B, Hq, Hkv, d, W)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_decode_sinks(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_sink), _ptr(v_sink), n_sink,
+                                 _ptr(o), _ptr(lse), _ptr(pos), B, Hq, Hkv, d, W, float(scale), _dtype_code(q),
+                                 _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "swa_decode_sinks")
     return o
 
 

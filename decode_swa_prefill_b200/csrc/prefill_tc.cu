@@ -171,7 +171,7 @@ __device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
     return q.active ? (q.te - q.ts) + n_glob : 0;
 }
 
-template <bool RING>
+template <bool RING, bool SINKS>
 __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, int n_mode1)
 {
     Work w;
@@ -266,7 +266,8 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs
                     w.q[x].te = hi_x[x] / BN - w.j_lo + 1;
                 }
         }
-        w.n_glob = (a.gidx != nullptr && a.g > 0) ? (a.g + BN - 1) / BN : 0;
+        // gathered tiles of global keys, or (SINKS) of the first g positions
+        w.n_glob = ((SINKS || a.gidx != nullptr) && a.g > 0) ? (a.g + BN - 1) / BN : 0;
     }
     w.hk = w.q[0].h / G;
     w.n_tiles = w.n_band + w.n_glob;
@@ -316,6 +317,16 @@ __device__ __forceinline__ void gather_rows(uint8_t *dst, int rows, int ch_bytes
     cp_async_wait_all();
 }
 
+// Gathered key tile of sink positions first .. first+nrows-1 (zeros after).
+template <int D>
+__device__ __forceinline__ void gather_sinks(uint8_t *dst, const __nv_bfloat16 *base, int first, int nrows, int b,
+                                             int T, int H, int head, int lane)
+{
+    gather_rows<D>(dst, BN, Cfg<D>::KCH, base, lane, [&](int r) -> const __nv_bfloat16 * {
+        return r < nrows ? base + (((long long)b * T + first + r) * H + head) * D : nullptr;
+    });
+}
+
 // Everything the softmax of one 64-key tile needs besides the scores.
 struct TileCtx {
     uint32_t s_addr;      // TMEM address of this warp's lanes of S[X][b]
@@ -330,7 +341,7 @@ struct TileCtx {
 // over the first 32 columns of the tile's TMEM buffer.  FULL: every key of
 // the tile is visible to every row of the warp (no masking, all chunks live),
 // the common case, compiled without any of the masking branches.
-template <bool FULL>
+template <bool FULL, bool SINKS>
 __device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillArgs &a, const int32_t *gb, float &m,
                                              float &l, bool &rescale, float &alpha, bool first)
 {
@@ -358,7 +369,11 @@ __device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillAr
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int gc = k.gc_base + cc * 32 + e;
-                    const bool keep = gc < a.g && !band_contains(k.i_row, __ldg(gb + gc), a.left, a.right);
+                    bool keep;
+                    if constexpr (SINKS) // sink position gc: up to the query's own position
+                        keep = gc < a.g && gc <= k.i_row && !band_contains(k.i_row, gc, a.left, a.right);
+                    else
+                        keep = gc < a.g && !band_contains(k.i_row, __ldg(gb + gc), a.left, a.right);
                     if (!keep) sr[cc * 32 + e] = -CUDART_INF_F;
                 }
             }
@@ -420,7 +435,7 @@ __device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillAr
 // (swa_prefill_chunk), compiled as its own kernel so that the other calls
 // keep 32-bit key positions, no ring branches and their four-map argument
 // list (two more tensor-map arguments alone cost those launches 2%).
-template <int D, bool RING>
+template <int D, bool RING, bool SINKS>
 __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                                             const CUtensorMap *tmO, const CUtensorMap *tmKr, const CUtensorMap *tmVr,
                                             const TcPrefillArgs &a, const RingArgs &ring, const int n_mode1)
@@ -435,7 +450,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const Work w = make_work<RING>(a, ring, n_mode1);
+    const Work w = make_work<RING, SINKS>(a, ring, n_mode1);
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -574,8 +589,12 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                                         key0, w.b);
                     }
                 } else {
-                    gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
-                                   gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                    if constexpr (SINKS)
+                        gather_sinks<D>(sK + st * C::KTILE, static_cast<const __nv_bfloat16 *>(a.k), gt * BN, nr, w.b,
+                                        a.T, a.Hkv, w.hk, lane);
+                    else
+                        gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
+                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->k_full[st]);
@@ -591,8 +610,12 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                                         key0, w.b);
                     }
                 } else {
-                    gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
-                                   gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                    if constexpr (SINKS)
+                        gather_sinks<D>(sV + st * C::KTILE, static_cast<const __nv_bfloat16 *>(a.v), gt * BN, nr, w.b,
+                                        a.T, a.Hkv, w.hk, lane);
+                    else
+                        gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
+                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->v_full[st]);
@@ -761,9 +784,9 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
             bool rescale_o;
             float alpha;
             if (interior && c_lo == 0 && c_hi == BN / 32 - 1)
-                softmax_tile<true>(k, a, gb, m, l, rescale_o, alpha, c == 0);
+                softmax_tile<true, SINKS>(k, a, gb, m, l, rescale_o, alpha, c == 0);
             else
-                softmax_tile<false>(k, a, gb, m, l, rescale_o, alpha, c == 0);
+                softmax_tile<false, SINKS>(k, a, gb, m, l, rescale_o, alpha, c == 0);
 
             // O rescale (rare): wait for the previous tile's PV, which
             // accumulates into O; this tile's PV waits for P
@@ -869,7 +892,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                           const TcPrefillArgs a, const int n_mode1)
 {
-    prefill_cta<D, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
+    prefill_cta<D, false, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
+}
+
+// Causal window plus attention sinks (a.gidx null, a.g sinks): the sink keys
+// form the gathered key tiles.
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    swa_prefill_sinks_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                             const TcPrefillArgs a, const int n_mode1)
+{
+    prefill_cta<D, false, true>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
 }
 
 template <int D>
@@ -879,7 +913,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
                             const TcPrefillArgs a, const RingArgs ring, const int n_mode1)
 {
-    prefill_cta<D, true>(&tmQ, &tmK, &tmV, &tmO, &tmKr, &tmVr, a, ring, n_mode1);
+    prefill_cta<D, true, false>(&tmQ, &tmK, &tmV, &tmO, &tmKr, &tmVr, a, ring, n_mode1);
 }
 
 // ------------------------------------------------------------------ host --
@@ -954,16 +988,21 @@ cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cu
         mkr = mk; // unused without a ring
         mvr = mv;
     }
-    static bool attr_set[64] = {};
+    // sinks: no global positions but g > 0 (causal window plus the first g
+    // positions)
+    const bool sinks = !RING && a.gidx == nullptr && a.g > 0;
+    static bool attr_set[64][2] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = RING ? cudaFuncSetAttribute(swa_prefill_ring_kernel<D>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
-                             : cudaFuncSetAttribute(swa_prefill_tc_kernel<D>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (dev < 64 && !attr_set[dev][sinks]) {
+        cudaError_t e = RING    ? cudaFuncSetAttribute(swa_prefill_ring_kernel<D>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                        : sinks ? cudaFuncSetAttribute(swa_prefill_sinks_kernel<D>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                                : cudaFuncSetAttribute(swa_prefill_tc_kernel<D>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev][sinks] = true;
     }
     const int G = a.Hq / a.Hkv;
     const bool pair_heads = (G % 2) == 0;
@@ -985,6 +1024,8 @@ cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cu
     if (grid == 0) return cudaSuccess;
     if (RING)
         swa_prefill_ring_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring, n_mode1);
+    else if (sinks)
+        swa_prefill_sinks_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, n_mode1);
     else
         swa_prefill_tc_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, n_mode1);
     return cudaGetLastError();

@@ -151,6 +151,8 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
         const long long ip = p0 + i;  // absolute position of the row
         const long long lo = max(0LL, ip - a.left);
         const long long hi = min(p0 + a.T - 1, ip + a.right);
+        if (!gb && a.g > 0)  // sinks older than the window
+            for (long long j = 0; j < min((long long)a.g, lo); ++j) visit(j);
         for (long long j = lo; j <= hi; ++j) visit(j);
         if (gb)
             for (int c = 0; c < a.g; ++c)
@@ -211,7 +213,7 @@ struct Ld<float> {
     __device__ __forceinline__ static void store(float *p, float x) { *p = x; }
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool SINKS>
 __global__ void __launch_bounds__(32 * DEC_WARPS)
     decode_kernel(DecodeArgs a)
 {
@@ -224,13 +226,25 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const long long p = a.pos[b];
     if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
-    const int chunk = (a.W + a.splits - 1) / a.splits;
+    // virtual slots: the sinks older than the window (positions < p-W+1)
+    // first, then the ring's filled slots
+    const int ns = SINKS ? (int)max(0LL, min((long long)a.n_sink, p - a.W + 1)) : 0;
+    const int chunk = (a.W + (SINKS ? a.n_sink : 0) + a.splits - 1) / a.splits;
     const int s_begin = split * chunk;
-    const int s_end = min(n_valid, s_begin + chunk);
+    const int s_end = min(ns + n_valid, s_begin + chunk);
 
     const T *qb = static_cast<const T *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
     const T *kb = static_cast<const T *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const T *vb = static_cast<const T *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+    const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
+    auto krow = [&](int sl) -> const T * {
+        if (SINKS && sl < ns) return static_cast<const T *>(a.ks) + sink0 + (long long)sl * D;
+        return kb + (long long)(sl - ns) * D;
+    };
+    auto vrow = [&](int sl) -> const T * {
+        if (SINKS && sl < ns) return static_cast<const T *>(a.vs) + sink0 + (long long)sl * D;
+        return vb + (long long)(sl - ns) * D;
+    };
 
     float q[G][EPL];
 #pragma unroll
@@ -254,8 +268,8 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
 #pragma unroll
         for (int n = 0; n < NB; ++n) {
             const int sl = min(base + n, s_end - 1); // clamp: masked below
-            Ld<T>::template row<EPL>(kb + (long long)sl * D + lane * EPL, kr[n]);
-            Ld<T>::template row<EPL>(vb + (long long)sl * D + lane * EPL, vr[n]);
+            Ld<T>::template row<EPL>(krow(sl) + lane * EPL, kr[n]);
+            Ld<T>::template row<EPL>(vrow(sl) + lane * EPL, vr[n]);
         }
         // partial dot products, value index n*G + g
         float v[32];
@@ -388,7 +402,7 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w)
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-template <int D, int G>
+template <int D, int G, bool SINKS>
 __global__ void __launch_bounds__(32 * DEC_WARPS)
     decode_bf16_kernel(DecodeArgs a)
 {
@@ -406,13 +420,25 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const long long p = a.pos[b];
     if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
-    const int chunk = (a.W + a.splits - 1) / a.splits;
+    // virtual slots: the sinks older than the window (positions < p-W+1)
+    // first, then the ring's filled slots
+    const int ns = SINKS ? (int)max(0LL, min((long long)a.n_sink, p - a.W + 1)) : 0;
+    const int chunk = (a.W + (SINKS ? a.n_sink : 0) + a.splits - 1) / a.splits;
     const int s_begin = split * chunk;
-    const int s_end = min(n_valid, s_begin + chunk);
+    const int s_end = min(ns + n_valid, s_begin + chunk);
 
     const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
+    const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
+    auto krow = [&](int sl) -> const __nv_bfloat16 * {
+        if (SINKS && sl < ns) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)sl * D;
+        return kb + (long long)(sl - ns) * D;
+    };
+    auto vrow = [&](int sl) -> const __nv_bfloat16 * {
+        if (SINKS && sl < ns) return static_cast<const __nv_bfloat16 *>(a.vs) + sink0 + (long long)sl * D;
+        return vb + (long long)(sl - ns) * D;
+    };
 
     uint4 q[G];
 #pragma unroll
@@ -432,8 +458,8 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
 #pragma unroll
         for (int n = 0; n < NBL; ++n) {
             const int sl = min(base + n * RPW + rgrp, s_end - 1); // clamp: masked below
-            kr[n] = __ldg(reinterpret_cast<const uint4 *>(kb + (long long)sl * D + part * 8));
-            vr[n] = __ldg(reinterpret_cast<const uint4 *>(vb + (long long)sl * D + part * 8));
+            kr[n] = __ldg(reinterpret_cast<const uint4 *>(krow(sl) + part * 8));
+            vr[n] = __ldg(reinterpret_cast<const uint4 *>(vrow(sl) + part * 8));
         }
         // partial dot products over this lane's 8 elements, index n*G + g
         float v[LPR];
@@ -587,10 +613,14 @@ template <typename T, int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
     dim3 grid(a.splits, a.Hkv, a.B);
-    if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8)
-        decode_bf16_kernel<D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
-    else
-        decode_kernel<T, D, G><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    const bool sinks = a.n_sink > 0;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8) {
+        if (sinks) decode_bf16_kernel<D, G, true><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+        else decode_bf16_kernel<D, G, false><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    } else {
+        if (sinks) decode_kernel<T, D, G, true><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+        else decode_kernel<T, D, G, false><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
     decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);

@@ -141,6 +141,33 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
     return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
 }
 
+swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink, int B,
+                             int T, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK) return st;
+    if (n_sink < 0) return SWA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return SWA_OK;
+    if (n_sink > T) n_sink = T;
+    const int left = W - 1 < T ? W - 1 : T;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == SWA_DTYPE_F32) {
+        // null global positions with g > 0: the first g positions are sinks
+        swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(o), lse, B, T, Hq, Hkv, d, left, 0,
+                              nullptr, n_sink, scale};
+        return from_cuda(swa::launch_prefill_f32(a, s));
+    }
+    swa::TcPrefillArgs a{};
+    a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv;
+    a.left = left; a.right = 0;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.lse = lse; a.gidx = nullptr; a.g = n_sink;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
+}
+
 swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *o, float *lse, const void *k_cache,
                              const void *v_cache, const int32_t *pos, int B, int n, int Hq, int Hkv, int d, int W,
                              float scale, swa_dtype dt, void *stream)
@@ -195,11 +222,17 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
     return swa::decode_workspace_bytes(B, Hq, Hkv, d, W);
 }
 
-swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
-                      const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
-                      void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// swa_decode and swa_decode_sinks (n_sink = 0: no sinks).
+swa_status decode_impl(const void *q, const void *k_cache, const void *v_cache, const void *k_sink,
+                       const void *v_sink, int n_sink, void *o, float *lse, const int32_t *pos, int B, int Hq, int Hkv,
+                       int d, int W, float scale, swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream)
 {
     if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (n_sink < 0) return SWA_ERR_INVALID_ARG;
     if (B < 0 || Hq < 1 || Hkv < 1 || W < 1 || d < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
     const int G = Hq / Hkv;
@@ -218,9 +251,34 @@ swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, v
     a.scale_log2 = scale * 1.4426950408889634f;
     a.splits = swa::decode_splits(B, Hq, Hkv, d, W);
     a.partial = static_cast<float *>(workspace);
+    if (n_sink > 0) {
+        if (!k_sink || !v_sink || !aligned(k_sink, 16) || !aligned(v_sink, 16)) return SWA_ERR_INVALID_ARG;
+        a.ks = k_sink; a.vs = v_sink; a.n_sink = n_sink;
+    }
     swa_status st = ctl(&a.ctl);
     if (st != SWA_OK) return st;
     return from_cuda(swa::launch_decode(dt == SWA_DTYPE_BF16, a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
+                      const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    return decode_impl(q, k_cache, v_cache, nullptr, nullptr, 0, o, lse, pos, B, Hq, Hkv, d, W, scale, dt, workspace,
+                       workspace_bytes, stream);
+}
+
+swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_cache, const void *k_sink,
+                            const void *v_sink, int n_sink, void *o, float *lse, const int32_t *pos, int B, int Hq,
+                            int Hkv, int d, int W, float scale, swa_dtype dt, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    return decode_impl(q, k_cache, v_cache, k_sink, v_sink, n_sink, o, lse, pos, B, Hq, Hkv, d, W, scale, dt,
+                       workspace, workspace_bytes, stream);
 }
 
 swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric, const int32_t *global_idx, int g,

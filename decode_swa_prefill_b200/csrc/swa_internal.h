@@ -53,6 +53,9 @@ struct RingArgs {
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s);
 
 // ---- SIMT kernels ----
+// Attention sinks in the prefill calls: gidx == null with g > 0 means the
+// first g positions of each sequence are keys every later query sees
+// (causal window only).
 struct F32PrefillArgs {
     const float *q, *k, *v;
     float *o, *lse;
@@ -79,6 +82,10 @@ struct DecodeArgs {
     float *partial;           // [B,Hq,S,d+2] when S > 1
     int splits;
     DeviceCtl ctl;
+    // attention sinks beside the ring: [B,Hkv,n_sink,d] caches of positions
+    // 0..n_sink-1 (n_sink = 0: none)
+    const void *ks, *vs;
+    int n_sink;
 };
 int decode_splits(int B, int Hq, int Hkv, int d, int W);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);

@@ -88,6 +88,22 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
                               swa_dtype dt, void *stream);
 
 /*
+ * Causal sliding-window prefill with attention sinks: the first n_sink tokens
+ * of each sequence stay visible to every later query beside its window
+ * (Ultralytics glossary, related-terms entry on attention sinks: StreamingLLM
+ * keeps them in the cache beside the window; robocikowo.com opening
+ * definition for the window).
+ *   o[b,i,h,:] = softmax-weighted sum over the keys j <= i with
+ *                j >= i-W+1 or j < n_sink (a sink inside the window counts
+ *                once)
+ *   n_sink >= 0 (0 is swa_prefill; n_sink >= T makes every row full causal).
+ *   Other arguments as swa_prefill.
+ */
+swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink,
+                             int B, int T, int Hq, int Hkv, int d, int W, float scale,
+                             swa_dtype dt, void *stream);
+
+/*
  * Causal prefill of a chunk of n new tokens that continues sequences whose
  * earlier tokens are already in the W-slot rings: token t of batch row b is
  * at position P = pos[b]+t and sees the keys at positions max(0,P-W+1) .. P
@@ -151,6 +167,23 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
                       const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
                       swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step over the ring plus attention sinks (Ultralytics glossary,
+ * related-terms entry on attention sinks).  The query at position P =
+ * pos[b] sees the ring's filled slots (the window, as in swa_decode) and
+ * the sinks older than the window, positions 0 .. min(n_sink, P-W+1)-1; a
+ * sink still inside the window is read once, from the ring.
+ *   k_sink, v_sink : [B,Hkv,n_sink,d], row j holding position j (written by
+ *                    the caller, e.g. swa_cache_append with W = n_sink while
+ *                    the positions are below n_sink); may be NULL when
+ *                    n_sink == 0
+ *   n_sink >= 0; other arguments, the workspace included, as swa_decode.
+ */
+swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_cache,
+                            const void *k_sink, const void *v_sink, int n_sink, void *o, float *lse,
+                            const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
+                            swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * swa_decode with no workspace argument, for callers that cannot allocate

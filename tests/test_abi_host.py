@@ -99,6 +99,20 @@ def test_prefill_chunk_rejects(lib):
     assert call(B=0, kc=NULL, vc=NULL, pos=NULL) == 0
 
 
+def test_sinks_reject(lib):
+    f = lib.swa_prefill_sinks
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, -1, 1, 16, 4, 2, 64, 8, 0.125, 1, NULL) == 1   # negative sinks
+    assert f(FAKE, FAKE, FAKE, FAKE, NULL, 2, 1, 16, 4, 2, 48, 8, 0.125, 1, NULL) == 2    # d
+    assert f(NULL, NULL, NULL, NULL, NULL, 2, 0, 16, 4, 2, 64, 8, 0.125, 1, NULL) == 0     # B == 0
+    g = lib.swa_decode_sinks
+    need = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
+    call = lambda ks=FAKE, vs=FAKE, n=4: g(FAKE, FAKE, FAKE, ks, vs, n, FAKE, NULL, FAKE, 64, 32, 8, 128, 4096,
+                                          0.088, 1, FAKE, need, NULL)
+    assert call(n=-1) == 1
+    assert call(ks=NULL) == 1
+    assert call(vs=MISALIGNED) == 1
+
+
 def test_append_rejects(lib):
     f = lib.swa_cache_append
     assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1      # no pos
