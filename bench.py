@@ -292,6 +292,7 @@ def gpu_arm(args, world, rank, local):
     e2e = e2e_arm(st, args, world, dev, step_flops)
     extra = tinymistral_arm(swa, dev, args)
     chunk = chunk_arm(swa, dev, args)
+    sinks = sinks_arm(swa, dev, args, load_peaks()[0])
 
     peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
@@ -321,6 +322,7 @@ def gpu_arm(args, world, rank, local):
             "append": {"us": round(avg["append"] * 1e3, 2)},
             "tinymistral_prefill": extra,
             "chunk_prefill": chunk,
+            "sinks": sinks,
             "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
@@ -401,6 +403,55 @@ def chunk_arm(swa, dev, args):
     tf = flops / (ms * 1e-3) / 1e12
     return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "flops": flops, "workload": w.name}
+
+
+def sink_pairs(T, W, s):
+    """In-window pairs of a causal window W plus s sinks: each row's window,
+    plus the sinks older than it."""
+    return causal_pairs(T, W) + sum(max(0, min(s, i - W + 1)) for i in range(T))
+
+
+def sinks_arm(swa, dev, args, peaks):
+    """Attention sinks (4 per sequence) beside the window: the Mistral-7B
+    prefill and decode configurations with sinks, not part of the step."""
+    n_sink = 4
+    w = wl.MISTRAL_PREFILL
+    q, k, v = (t.to(dev) for t in wl.prefill_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.dtype, w.seed))
+    o = torch.empty_like(q)
+    pf = sink_pairs(w.T, w.W, n_sink) * w.B * w.Hq * 4 * w.d
+    wd = wl.MISTRAL_DECODE
+    dq, kc, vc, _, _, pos = wl.decode_inputs(wd.B, wd.Hq, wd.Hkv, wd.d, wd.W, wd.dtype, wd.seed, wd.pos_lo,
+                                             wd.pos_hi)
+    _, ks, vs, _, _, _ = wl.decode_inputs(wd.B, wd.Hq, wd.Hkv, wd.d, n_sink, wd.dtype, wd.seed + 1, 0, 1)
+    dq, kc, vc, ks, vs, pos = (t.to(dev) for t in (dq, kc, vc, ks, vs, pos))
+    do = torch.empty_like(dq)
+    ws = torch.empty(max(1, swa.swa_decode_workspace_bytes(wd.B, wd.Hq, wd.Hkv, wd.d, wd.W)), dtype=torch.uint8,
+                     device=dev)
+    dbytes = wd.B * wd.Hkv * (wd.W + n_sink) * wd.d * 2 * 2
+    res = {}
+    for name, fn, work in (
+            ("prefill", lambda: swa.swa_prefill_sinks(q, k, v, w.W, n_sink, o=o), pf),
+            ("decode", lambda: swa.swa_decode_sinks(dq, kc, vc, ks, vs, pos, o=do, workspace=ws), dbytes)):
+        times = []
+        for i in range(args.warmup + max(10, args.steps // 2)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        ms = sum(times) / len(times)
+        if name == "prefill":
+            tf = work / (ms * 1e-3) / 1e12
+            res[name] = {"tflops": round(tf, 2), "ms": round(ms, 4),
+                         "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4)}
+        else:
+            gbs = work / (ms * 1e-3) / 1e9
+            res[name] = {"gbs": round(gbs, 1), "us": round(ms * 1e3, 2),
+                         "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4)}
+    res["n_sink"] = n_sink
+    return res
 
 
 def e2e_arm(st, args, world, dev, step_flops):

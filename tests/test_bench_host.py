@@ -32,6 +32,11 @@ def test_chunk_pairs_match_oracle(n, W, p0):
     assert bench.chunk_pairs(n, W, p0) == oracle.count_pairs(p0 + n, W) - oracle.count_pairs(p0, W)
 
 
+@pytest.mark.parametrize("T,W,s", [(16, 4, 2), (30, 7, 0), (9, 20, 4), (100, 10, 100), (64, 1, 3)])
+def test_sink_pairs_match_oracle(T, W, s):
+    assert bench.sink_pairs(T, W, s) == oracle.count_pairs_sinks(T, W, s)
+
+
 def test_step_accounting_totals():
     acc = bench.step_accounting(wl.make(wl.LONGFORMER))
     assert acc["f_prefill"] == 125_831_168 * 32 * 4 * 128
