@@ -226,24 +226,25 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const long long p = a.pos[b];
     if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
-    // virtual slots: the sinks older than the window (positions < p-W+1)
-    // first, then the ring's filled slots
+    // virtual slots: the ring's filled slots, then the sinks older than the
+    // window (positions < p-W+1), which the last split takes on top of its
+    // share of the ring (the ring keeps the plain decode's split boundaries)
     const int ns = SINKS ? (int)max(0LL, min((long long)a.n_sink, p - a.W + 1)) : 0;
-    const int chunk = (a.W + (SINKS ? a.n_sink : 0) + a.splits - 1) / a.splits;
+    const int chunk = (a.W + a.splits - 1) / a.splits;
     const int s_begin = split * chunk;
-    const int s_end = min(ns + n_valid, s_begin + chunk);
+    const int s_end = (SINKS && split == a.splits - 1) ? n_valid + ns : min(n_valid, s_begin + chunk);
 
     const T *qb = static_cast<const T *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
     const T *kb = static_cast<const T *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const T *vb = static_cast<const T *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
     auto krow = [&](int sl) -> const T * {
-        if (SINKS && sl < ns) return static_cast<const T *>(a.ks) + sink0 + (long long)sl * D;
-        return kb + (long long)(sl - ns) * D;
+        if (SINKS && sl >= n_valid) return static_cast<const T *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
+        return kb + (long long)sl * D;
     };
     auto vrow = [&](int sl) -> const T * {
-        if (SINKS && sl < ns) return static_cast<const T *>(a.vs) + sink0 + (long long)sl * D;
-        return vb + (long long)(sl - ns) * D;
+        if (SINKS && sl >= n_valid) return static_cast<const T *>(a.vs) + sink0 + (long long)(sl - n_valid) * D;
+        return vb + (long long)sl * D;
     };
 
     float q[G][EPL];
@@ -420,24 +421,25 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const long long p = a.pos[b];
     if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
-    // virtual slots: the sinks older than the window (positions < p-W+1)
-    // first, then the ring's filled slots
+    // virtual slots: the ring's filled slots, then the sinks older than the
+    // window (positions < p-W+1), which the last split takes on top of its
+    // share of the ring (the ring keeps the plain decode's split boundaries)
     const int ns = SINKS ? (int)max(0LL, min((long long)a.n_sink, p - a.W + 1)) : 0;
-    const int chunk = (a.W + (SINKS ? a.n_sink : 0) + a.splits - 1) / a.splits;
+    const int chunk = (a.W + a.splits - 1) / a.splits;
     const int s_begin = split * chunk;
-    const int s_end = min(ns + n_valid, s_begin + chunk);
+    const int s_end = (SINKS && split == a.splits - 1) ? n_valid + ns : min(n_valid, s_begin + chunk);
 
     const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) + ((long long)b * Hq + (long long)hk * G) * D;
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
     auto krow = [&](int sl) -> const __nv_bfloat16 * {
-        if (SINKS && sl < ns) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)sl * D;
-        return kb + (long long)(sl - ns) * D;
+        if (SINKS && sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
+        return kb + (long long)sl * D;
     };
     auto vrow = [&](int sl) -> const __nv_bfloat16 * {
-        if (SINKS && sl < ns) return static_cast<const __nv_bfloat16 *>(a.vs) + sink0 + (long long)sl * D;
-        return vb + (long long)(sl - ns) * D;
+        if (SINKS && sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.vs) + sink0 + (long long)(sl - n_valid) * D;
+        return vb + (long long)sl * D;
     };
 
     uint4 q[G];
