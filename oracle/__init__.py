@@ -64,6 +64,13 @@ def _load():
         lib.oracle_swa_decode_sinks.argtypes = [p, p, p, p, p, p, p, p, c_long, c_long, c_long, c_long,
                                                 c_long, c_long, c_double]
         lib.oracle_swa_decode_sinks.restype = c_int
+        lib.oracle_dilated_allowed.argtypes = [c_long, c_long, c_long, c_long, c_long, c_int]
+        lib.oracle_dilated_allowed.restype = c_int
+        lib.oracle_count_pairs_dilated.argtypes = [c_long, c_long, c_long, c_int]
+        lib.oracle_count_pairs_dilated.restype = ctypes.c_longlong
+        lib.oracle_swa_prefill_dilated.argtypes = [p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
+                                                   c_long, c_long, c_int, c_double, p, c_long, c_int]
+        lib.oracle_swa_prefill_dilated.restype = c_int
         _lib = lib
     return _lib
 
@@ -275,3 +282,33 @@ def swa_decode_sinks(q, k_cache, v_cache, k_sink, v_sink, pos, scale=None):
     if rc != 0:
         raise ValueError("negative position")
     return o, lse
+
+
+# ---------------------------------------------------------------- dilated --
+
+def dilated_allowed(i, j, T, W, dil, mode=CAUSAL):
+    """Dilated window (aivaro.ru section 4.2): causal keys i - dil*m,
+    m = 0..W-1; symmetric keys i + dil*m, |m| <= W//2."""
+    return bool(_load().oracle_dilated_allowed(i, j, T, W, dil, mode))
+
+
+def count_pairs_dilated(T, W, dil, mode=CAUSAL):
+    return int(_load().oracle_count_pairs_dilated(T, W, dil, mode))
+
+
+def swa_prefill_dilated(q, k, v, W, dil, mode=CAUSAL, scale=None, rows=None, nthreads=None):
+    """Dilated sliding-window prefill (aivaro.ru section 4.2); shapes and row
+    selection as swa_prefill."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = _rows_arg(rows, B, Hq, T)
+    o = np.zeros((len(r), d)); lse = np.zeros(len(r))
+    rc = _load().oracle_swa_prefill_dilated(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
+                                            int(dil), int(mode), float(scale), _ptr(r), len(r),
+                                            nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("bad dilation or mode")
+    return _unflatten(o, lse, r, rows is None, B, T, Hq, d)

@@ -80,6 +80,30 @@ int oracle_sink_allowed(long i, long j, long T, long W, long s)
     return j >= i - W + 1 || j < s;
 }
 
+/* Dilated window [P2 s.4.2: instead of all W neighbours, every dil-th token
+ * is taken, which widens the span without more keys].  Causal: keys
+ * i - dil*m for m = 0..W-1; symmetric: keys i + dil*m for |m| <= W/2.  The
+ * page's worked example is garbled (its key count and span disagree); the
+ * reading taken keeps W keys (W/2 per side) and stretches the span by dil. */
+int oracle_dilated_allowed(long i, long j, long T, long W, long dil, int mode)
+{
+    if (j < 0 || j >= T || i < 0 || i >= T || dil < 1) return 0;
+    const long diff = i - j;
+    if (diff % dil != 0) return 0;
+    const long m = diff / dil;
+    if (mode == ORACLE_CAUSAL) return m >= 0 && m <= W - 1;
+    const long h = W / 2;
+    return m >= -h && m <= h;
+}
+
+long long oracle_count_pairs_dilated(long T, long W, long dil, int mode)
+{
+    long long n = 0;
+    for (long i = 0; i < T; i++)
+        for (long j = 0; j < T; j++) n += oracle_dilated_allowed(i, j, T, W, dil, mode);
+    return n;
+}
+
 /* Pairs a causal window with s sinks allows. */
 long long oracle_count_pairs_sinks(long T, long W, long s)
 {
@@ -202,6 +226,7 @@ typedef struct {
     const int32_t *gidx; /* [B,g] or NULL */
     long g;
     long sinks;          /* causal window plus the first `sinks` tokens (mode ORACLE_SINKS) */
+    long dil;            /* dilation (> 1: modes ORACLE_DILATED_*) */
     double scale;
     const int64_t *rows; /* flattened (b*Hq + h)*T + i */
     long nrows;
@@ -219,8 +244,10 @@ static void prefill_one(prefill_job *J, long r, const double **kr, const double 
     const int32_t *gb = J->gidx ? J->gidx + b * J->g : NULL;
     long n = 0;
     for (long j = 0; j < J->T; j++) {
-        const int ok = J->mode == ORACLE_SINKS ? oracle_sink_allowed(i, j, J->T, J->W, J->sinks)
-                                               : oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0);
+        int ok;
+        if (J->mode == ORACLE_SINKS) ok = oracle_sink_allowed(i, j, J->T, J->W, J->sinks);
+        else if (J->dil > 1) ok = oracle_dilated_allowed(i, j, J->T, J->W, J->dil, J->mode);
+        else ok = oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0);
         if (!ok) continue;
         kr[n] = J->k + ((b * J->T + j) * J->Hkv + hk) * J->d;
         vr[n] = J->v + ((b * J->T + j) * J->Hkv + hk) * J->d;
@@ -271,7 +298,7 @@ int oracle_swa_prefill(const double *q, const double *k, const double *v, double
                        long B, long T, long Hq, long Hkv, long d, long W, double scale,
                        const int64_t *rows, long nrows, int nthreads)
 {
-    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_CAUSAL, NULL, 0, 0, scale, rows, nrows};
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_CAUSAL, NULL, 0, 0, 1, scale, rows, nrows};
     return run_prefill(&J, nthreads);
 }
 
@@ -283,7 +310,7 @@ int oracle_swa_prefill_global(const double *q, const double *k, const double *v,
                               long B, long T, long Hq, long Hkv, long d, long W, double scale,
                               const int64_t *rows, long nrows, int nthreads)
 {
-    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SYMMETRIC, g > 0 ? gidx : NULL, g, 0, scale, rows, nrows};
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SYMMETRIC, g > 0 ? gidx : NULL, g, 0, 1, scale, rows, nrows};
     return run_prefill(&J, nthreads);
 }
 
@@ -293,7 +320,18 @@ int oracle_swa_prefill_sinks(const double *q, const double *k, const double *v, 
                              long B, long T, long Hq, long Hkv, long d, long W, long s, double scale,
                              const int64_t *rows, long nrows, int nthreads)
 {
-    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SINKS, NULL, 0, s, scale, rows, nrows};
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, ORACLE_SINKS, NULL, 0, s, 1, scale, rows, nrows};
+    return run_prefill(&J, nthreads);
+}
+
+/* Dilated window, causal (mode 0) or symmetric (mode 1) [P2 s.4.2]; the
+ * keys of each row are those oracle_dilated_allowed admits. */
+int oracle_swa_prefill_dilated(const double *q, const double *k, const double *v, double *o, double *lse,
+                               long B, long T, long Hq, long Hkv, long d, long W, long dil, int mode,
+                               double scale, const int64_t *rows, long nrows, int nthreads)
+{
+    if (dil < 1 || (mode != ORACLE_CAUSAL && mode != ORACLE_SYMMETRIC)) return -1;
+    prefill_job J = {q, k, v, o, lse, B, T, Hq, Hkv, d, W, mode, NULL, 0, 0, dil, scale, rows, nrows};
     return run_prefill(&J, nthreads);
 }
 
