@@ -16,8 +16,9 @@ import torch
 
 __all__ = [
     "SwaError", "load", "library_path", "EXPORTED",
-    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_cache_append",
-    "swa_decode", "swa_decode_sinks", "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
+    "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_prefill_dilated",
+    "swa_prefill_dilated_workspace_bytes", "swa_cache_append", "swa_decode", "swa_decode_sinks",
+    "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
     "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
 
@@ -30,6 +31,7 @@ SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 # every symbol include/swa.h declares
 EXPORTED = [
     "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
+    "swa_prefill_dilated", "swa_prefill_dilated_workspace_bytes",
     "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
     "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
@@ -58,6 +60,9 @@ def load():
     lib.swa_prefill_global.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
     lib.swa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.swa_prefill_sinks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_prefill_dilated.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
+    lib.swa_prefill_dilated_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
+    lib.swa_prefill_dilated_workspace_bytes.restype = ctypes.c_size_t
     lib.swa_decode_sinks.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -72,6 +77,7 @@ def load():
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
+                 "swa_prefill_dilated",
                  "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
         getattr(lib, name).restype = ctypes.c_int
@@ -129,6 +135,33 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
     st = load().swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
                             float(scale), _dtype_code(q), _stream(stream))
     _check(st, "swa_prefill")
+    return o
+
+
+def swa_prefill_dilated_workspace_bytes(B, T, Hq, Hkv, d, dil, dtype=torch.bfloat16, with_lse=False):
+    code = SWA_DTYPE_BF16 if dtype == torch.bfloat16 else SWA_DTYPE_F32
+    return int(load().swa_prefill_dilated_workspace_bytes(B, T, Hq, Hkv, d, dil, code, int(bool(with_lse))))
+
+
+def swa_prefill_dilated(q, k, v, W, dil, symmetric=False, scale=None, o=None, lse=None, workspace=None,
+                        stream=None):
+    """Dilated window (every dil-th key, W keys, or W//2 per side when
+    symmetric); the workspace is allocated here when not given."""
+    _dev_contig(q, k, v, o, lse, workspace)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, T, Hkv, d) and v.shape == k.shape, "k/v shape")
+    if o is None:
+        o = torch.empty_like(q)
+    need = swa_prefill_dilated_workspace_bytes(B, T, Hq, Hkv, d, dil, q.dtype, lse is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_dilated(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(dil), int(bool(symmetric)),
+                                    B, T, Hq, Hkv, d, W, float(scale), _dtype_code(q), _ptr(workspace), ws_bytes,
+                                    _stream(stream))
+    _check(st, "swa_prefill_dilated")
     return o
 
 

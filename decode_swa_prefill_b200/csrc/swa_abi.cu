@@ -71,6 +71,42 @@ swa_status check_prefill(const void *q, const void *k, const void *v, const void
     return SWA_OK;
 }
 
+// Workspace layout of a dilated prefill: per residue group, the permuted q,
+// k, v, o and (when asked for) lse, each at a 256-byte boundary.
+struct DilatedPlan {
+    int ng = 0;
+    swa::DilateGroup g[2];
+    size_t q[2], k[2], v[2], o[2], l[2];
+    size_t total = 0;
+};
+
+DilatedPlan dilated_plan(int B, int T, int Hq, int Hkv, int d, int dil, swa_dtype dt, bool with_lse)
+{
+    DilatedPlan p;
+    const int a = T % dil, lo = T / dil;
+    const int row16 = (int)(d * elt_size(dt) / 16);
+    auto add = [&](int r0, int n, int L) {
+        if (n <= 0 || L <= 0) return;
+        swa::DilateGroup g{B, T, 0, row16, dil, r0, n, L};
+        const size_t rows = (size_t)B * n * L;
+        auto take = [&](size_t bytes) {
+            const size_t off = p.total;
+            p.total += (bytes + 255) / 256 * 256;
+            return off;
+        };
+        const size_t rb = (size_t)d * elt_size(dt);
+        p.q[p.ng] = take(rows * Hq * rb);
+        p.k[p.ng] = take(rows * Hkv * rb);
+        p.v[p.ng] = take(rows * Hkv * rb);
+        p.o[p.ng] = take(rows * Hq * rb);
+        p.l[p.ng] = with_lse ? take(rows * Hq * sizeof(float)) : 0;
+        p.g[p.ng++] = g;
+    };
+    add(0, a, lo + 1);      // residues with one row more
+    add(a, dil - a, lo);
+    return p;
+}
+
 }  // namespace
 
 int swa::device_ctl(swa::DeviceCtl *c) { return ctl(c) == SWA_OK ? 0 : 1; }
@@ -139,6 +175,68 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
     a.q = q; a.k = k; a.v = v; a.o = o;
     if ((st = ctl(&a.ctl)) != SWA_OK) return st;
     return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
+}
+
+size_t swa_prefill_dilated_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int dil, swa_dtype dt, int with_lse)
+{
+    if (!valid_dtype(dt) || B <= 0 || T <= 0 || Hq < 1 || Hkv < 1 || d < 1 || dil <= 1) return 0;
+    return dilated_plan(B, T, Hq, Hkv, d, dil, dt, with_lse != 0).total;
+}
+
+swa_status swa_prefill_dilated(const void *q, const void *k, const void *v, void *o, float *lse, int dil,
+                               int symmetric, int B, int T, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
+                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK) return st;
+    if (dil < 1 || (symmetric != 0 && symmetric != 1)) return SWA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return SWA_OK;
+    if (dil == 1)
+        return symmetric ? swa_prefill_global(q, k, v, o, lse, nullptr, 0, B, T, Hq, Hkv, d, W, scale, dt, stream)
+                         : swa_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt, stream);
+    const DilatedPlan p = dilated_plan(B, T, Hq, Hkv, d, dil, dt, lse != nullptr);
+    if (!workspace || workspace_bytes < p.total || !aligned(workspace, 256)) return SWA_ERR_INVALID_ARG;
+    if ((long long)B * dil > (1 << 30)) return SWA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    swa::DeviceCtl c;
+    if ((st = ctl(&c)) != SWA_OK) return st;
+    for (int i = 0; i < p.ng; ++i) {
+        swa::DilateGroup gq = p.g[i], gk = p.g[i];
+        gq.H = Hq;
+        gk.H = Hkv;
+        cudaError_t e;
+        if ((e = swa::launch_dilate_rows(q, ws + p.q[i], gq, 1, s)) != cudaSuccess) return from_cuda(e);
+        if ((e = swa::launch_dilate_rows(k, ws + p.k[i], gk, 1, s)) != cudaSuccess) return from_cuda(e);
+        if ((e = swa::launch_dilate_rows(v, ws + p.v[i], gk, 1, s)) != cudaSuccess) return from_cuda(e);
+        // the sub-sequences as a batch of B*n sequences of L rows
+        const int Bg = B * gq.n, L = gq.L;
+        const int left = symmetric ? (W / 2 < L ? W / 2 : L) : (W - 1 < L ? W - 1 : L);
+        const int right = symmetric ? left : 0;
+        float *lse_g = lse ? reinterpret_cast<float *>(ws + p.l[i]) : nullptr;
+        if (dt == SWA_DTYPE_F32) {
+            swa::F32PrefillArgs a{reinterpret_cast<const float *>(ws + p.q[i]), reinterpret_cast<const float *>(ws + p.k[i]),
+                                  reinterpret_cast<const float *>(ws + p.v[i]), reinterpret_cast<float *>(ws + p.o[i]),
+                                  lse_g, Bg, L, Hq, Hkv, d, left, right, nullptr, 0, scale};
+            e = swa::launch_prefill_f32(a, s);
+        } else {
+            swa::TcPrefillArgs a{};
+            a.B = Bg; a.T = L; a.Hq = Hq; a.Hkv = Hkv;
+            a.left = left; a.right = right;
+            a.scale_log2 = scale * 1.4426950408889634f;
+            a.lse = lse_g; a.gidx = nullptr; a.g = 0;
+            a.q = ws + p.q[i]; a.k = ws + p.k[i]; a.v = ws + p.v[i]; a.o = ws + p.o[i];
+            a.ctl = c;
+            e = swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s);
+        }
+        if (e != cudaSuccess) return from_cuda(e);
+        if ((e = swa::launch_dilate_rows(ws + p.o[i], o, gq, 0, s)) != cudaSuccess) return from_cuda(e);
+        if (lse) {
+            gq.H = Hq;
+            if ((e = swa::launch_dilate_lse(lse_g, lse, gq, s)) != cudaSuccess) return from_cuda(e);
+        }
+    }
+    return SWA_OK;
 }
 
 swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink, int B,

@@ -107,6 +107,17 @@ cudaError_t launch_mask_export(uint8_t *mask, int T, int left, int right, const 
 
 cudaError_t launch_debug_expire_wait(const DeviceCtl &ctl, cudaStream_t s);
 
+// ---- dilated window: residue-major sub-sequence permutations ----
+// Group of residues r0 .. r0+n-1 of a [B,T,H,...] tensor, each a sub-sequence
+// of L rows at positions r0 + rr + t*dil.
+struct DilateGroup {
+    int B, T, H;
+    int row16;   // 16-byte units per row (row bytes / 16)
+    int dil, r0, n, L;
+};
+cudaError_t launch_dilate_rows(const void *src, void *dst, const DilateGroup &g, int to_group, cudaStream_t s);
+cudaError_t launch_dilate_lse(const float *src, float *dst, const DilateGroup &g, cudaStream_t s);
+
 // Fills the current device's status-word address and the wait limit; 0 on
 // success.
 int device_ctl(DeviceCtl *c);

@@ -88,6 +88,28 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
                               swa_dtype dt, void *stream);
 
 /*
+ * Dilated sliding-window prefill (aivaro.ru section 4.2: instead of all
+ * neighbours, every dil-th token, which widens the span without more keys).
+ *   symmetric = 0: query i sees keys i - dil*m, m = 0 .. W-1 (j >= 0)
+ *   symmetric = 1: query i sees keys i + dil*m, |m| <= W/2 (0 <= j < T)
+ *   The page's worked example is inconsistent (its key count and span
+ *   disagree); the window keeps W keys (W/2 per side) and its span grows by
+ *   dil.  dil = 1 is swa_prefill (symmetric: swa_prefill_global without
+ *   globals) and needs no workspace.
+ *   Such a window only pairs positions with equal residues modulo dil, so the
+ *   call permutes q, k, v into the dil strided sub-sequences, runs the plain
+ *   window on them and permutes o (and lse) back.
+ *   workspace : device scratch of swa_prefill_dilated_workspace_bytes(...)
+ *               bytes, 256-byte aligned; calls sharing it must not overlap.
+ *   Other arguments as swa_prefill.
+ */
+size_t swa_prefill_dilated_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int dil, swa_dtype dt,
+                                           int with_lse);
+swa_status swa_prefill_dilated(const void *q, const void *k, const void *v, void *o, float *lse, int dil,
+                               int symmetric, int B, int T, int Hq, int Hkv, int d, int W, float scale,
+                               swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Causal sliding-window prefill with attention sinks: the first n_sink tokens
  * of each sequence stay visible to every later query beside its window
  * (Ultralytics glossary, related-terms entry on attention sinks: StreamingLLM

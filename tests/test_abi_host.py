@@ -113,6 +113,20 @@ def test_sinks_reject(lib):
     assert call(vs=MISALIGNED) == 1
 
 
+def test_dilated_rejects(lib):
+    f = lib.swa_prefill_dilated
+    need = lib.swa_prefill_dilated_workspace_bytes(2, 300, 8, 2, 64, 3, 1, 0)
+    assert need > 0
+    assert lib.swa_prefill_dilated_workspace_bytes(2, 300, 8, 2, 64, 1, 1, 0) == 0   # dil 1: none
+    call = lambda dil=3, sym=0, ws=FAKE, wsb=need: f(FAKE, FAKE, FAKE, FAKE, NULL, dil, sym, 2, 300, 8, 2, 64, 16,
+                                                     0.125, 1, ws, wsb, NULL)
+    assert call(dil=0) == 1
+    assert call(sym=2) == 1
+    assert call(ws=NULL) == 1
+    assert call(wsb=need - 1) == 1
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 1      # workspace needs 256-byte alignment
+
+
 def test_append_rejects(lib):
     f = lib.swa_cache_append
     assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1      # no pos
