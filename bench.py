@@ -293,6 +293,7 @@ def gpu_arm(args, world, rank, local):
     extra = tinymistral_arm(swa, dev, args)
     chunk = chunk_arm(swa, dev, args)
     sinks = sinks_arm(swa, dev, args, load_peaks()[0])
+    dilated = dilated_arm(swa, dev, args, load_peaks()[0])
 
     peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
@@ -323,6 +324,7 @@ def gpu_arm(args, world, rank, local):
             "tinymistral_prefill": extra,
             "chunk_prefill": chunk,
             "sinks": sinks,
+            "dilated": dilated,
             "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
@@ -403,6 +405,39 @@ def chunk_arm(swa, dev, args):
     tf = flops / (ms * 1e-3) / 1e12
     return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "flops": flops, "workload": w.name}
+
+
+def dilated_pairs(T, W, dil, symmetric):
+    """In-window pairs of a dilated window (W keys with stride dil, or W//2
+    per side)."""
+    if not symmetric:
+        return sum(min(W, i // dil + 1) for i in range(T))
+    h = W // 2
+    return sum(min(h, i // dil) + min(h, (T - 1 - i) // dil) + 1 for i in range(T))
+
+
+def dilated_arm(swa, dev, args, peaks):
+    """Dilated symmetric window (Longformer shapes without global tokens,
+    dilation 2), timed with its two permutations: not part of the step."""
+    w, dil = wl.LONGFORMER, 2
+    q, k, v = (t.to(dev) for t in wl.prefill_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.dtype, w.seed))
+    o = torch.empty_like(q)
+    ws = torch.empty(swa.swa_prefill_dilated_workspace_bytes(w.B, w.T, w.Hq, w.Hkv, w.d, dil), dtype=torch.uint8,
+                     device=dev)
+    flops = dilated_pairs(w.T, w.W, dil, True) * w.B * w.Hq * 4 * w.d
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill_dilated(q, k, v, w.W, dil, symmetric=True, o=o, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "flops": flops, "dil": dil, "workload": "longformer_B8_T4096_h12_d64_W512_dil2_symmetric"}
 
 
 def sink_pairs(T, W, s):

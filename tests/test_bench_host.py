@@ -37,6 +37,12 @@ def test_sink_pairs_match_oracle(T, W, s):
     assert bench.sink_pairs(T, W, s) == oracle.count_pairs_sinks(T, W, s)
 
 
+@pytest.mark.parametrize("T,W,dil,sym", [(16, 4, 2, False), (30, 6, 3, True), (9, 20, 4, False), (40, 2, 7, True)])
+def test_dilated_pairs_match_oracle(T, W, dil, sym):
+    mode = oracle.SYMMETRIC if sym else oracle.CAUSAL
+    assert bench.dilated_pairs(T, W, dil, sym) == oracle.count_pairs_dilated(T, W, dil, mode)
+
+
 def test_step_accounting_totals():
     acc = bench.step_accounting(wl.make(wl.LONGFORMER))
     assert acc["f_prefill"] == 125_831_168 * 32 * 4 * 128
