@@ -312,3 +312,25 @@ def swa_prefill_dilated(q, k, v, W, dil, mode=CAUSAL, scale=None, rows=None, nth
     if rc != 0:
         raise ValueError("bad dilation or mode")
     return _unflatten(o, lse, r, rows is None, B, T, Hq, d)
+
+
+# ----------------------------------------------------------------- varlen --
+
+def swa_prefill_varlen(q, k, v, cu_seqlens, W, scale=None, nthreads=None):
+    """Causal window over packed sequences: q [total,Hq,d], k/v
+    [total,Hkv,d]; sequence b holds rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+    and attends within itself only (every sequence is its own causal
+    prefill, robocikowo.com opening definition).  Returns o [total,Hq,d] and
+    lse [Hq,total]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu = [int(x) for x in _i32(cu_seqlens)]
+    total, Hq, d = q.shape
+    o = np.zeros((total, Hq, d)); lse = np.zeros((Hq, total))
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        if hi <= lo:
+            continue
+        ob, lb = swa_prefill(q[None, lo:hi], k[None, lo:hi], v[None, lo:hi], W, scale=scale, nthreads=nthreads)
+        o[lo:hi] = ob[0]
+        lse[:, lo:hi] = lb[0]
+    return o, lse
