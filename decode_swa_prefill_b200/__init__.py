@@ -17,7 +17,8 @@ import torch
 __all__ = [
     "SwaError", "load", "library_path", "EXPORTED",
     "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_prefill_dilated",
-    "swa_prefill_dilated_workspace_bytes", "swa_cache_append", "swa_decode", "swa_decode_sinks",
+    "swa_prefill_dilated_workspace_bytes", "swa_prefill_varlen", "swa_cache_append", "swa_decode",
+    "swa_decode_sinks",
     "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
     "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
 ]
@@ -31,7 +32,7 @@ SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 # every symbol include/swa.h declares
 EXPORTED = [
     "swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
-    "swa_prefill_dilated", "swa_prefill_dilated_workspace_bytes",
+    "swa_prefill_dilated", "swa_prefill_dilated_workspace_bytes", "swa_prefill_varlen",
     "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
     "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
@@ -63,6 +64,7 @@ def load():
     lib.swa_prefill_dilated.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_prefill_dilated_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
     lib.swa_prefill_dilated_workspace_bytes.restype = ctypes.c_size_t
+    lib.swa_prefill_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
     lib.swa_decode_sinks.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -77,7 +79,7 @@ def load():
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
-                 "swa_prefill_dilated",
+                 "swa_prefill_dilated", "swa_prefill_varlen",
                  "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
         getattr(lib, name).restype = ctypes.c_int
@@ -135,6 +137,27 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
     st = load().swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, d, W,
                             float(scale), _dtype_code(q), _stream(stream))
     _check(st, "swa_prefill")
+    return o
+
+
+def swa_prefill_varlen(q, k, v, cu_seqlens, W, max_seqlen=None, scale=None, o=None, lse=None, stream=None):
+    """Causal window over packed sequences q [total,Hq,d], k/v [total,Hkv,d];
+    cu_seqlens int32 [nseq+1] on the device.  max_seqlen (the longest
+    sequence) is read from cu_seqlens when not given."""
+    _dev_contig(q, k, v, o, lse, cu_seqlens)
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    _need(k.shape == (total, Hkv, d) and v.shape == k.shape, "k/v shape")
+    _need(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1, "cu_seqlens int32 [nseq+1]")
+    nseq = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if nseq > 0 else 0
+    if o is None:
+        o = torch.empty_like(q)
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), nseq, total,
+                                   int(max_seqlen), Hq, Hkv, d, W, float(scale), _dtype_code(q), _stream(stream))
+    _check(st, "swa_prefill_varlen")
     return o
 
 

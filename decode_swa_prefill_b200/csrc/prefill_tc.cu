@@ -171,13 +171,15 @@ __device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
     return q.active ? (q.te - q.ts) + n_glob : 0;
 }
 
-template <bool RING, bool SINKS>
-__device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, int n_mode1)
+template <bool RING, bool SINKS, bool VARLEN>
+__device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl,
+                                          int n_mode1)
 {
     Work w;
     const int G = a.Hq / a.Hkv;
     const bool pair_heads = (G % 2) == 0;
-    const int nqt = (a.T + BM - 1) / BM;
+    // query tiles per sequence (the longest one for packed sequences)
+    const int nqt = ((VARLEN ? vl.max_len : a.T) + BM - 1) / BM;
     const int nkt = (a.T + BN - 1) / BN;
     const int ngt = (a.g + BM - 1) / BM;
     int bid = blockIdx.x;
@@ -247,14 +249,26 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs
                     w.q[x].te = (int)(hi_x[x] / BN) - w.j_lo + 1;
                 }
         } else {
+            // sequence length (a packed sequence: its own; tiles past it idle)
+            int TT = a.T;
+            if constexpr (VARLEN) {
+                // an inconsistent entry (decreasing, past the rows, longer
+                // than max_len) makes the sequence empty; the CTA reports it
+                const int c0 = vl.cu[w.b], c1 = vl.cu[w.b + 1];
+                TT = (c0 < 0 || c1 < c0 || c1 > a.T || c1 - c0 > vl.max_len) ? 0 : c1 - c0;
+                for (int x = 0; x < 2; ++x) {
+                    if (w.q[x].m0 >= TT) w.q[x].active = false;
+                    w.q[x].nrows = min(BM, TT - w.q[x].m0);
+                }
+            }
             w.p0 = 0;
-            w.kend = a.T;
-            int lo = a.T, hi = -1;
+            w.kend = TT;
+            int lo = TT, hi = -1;
             int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
             for (int x = 0; x < 2; ++x) {
                 if (!w.q[x].active) continue;
                 lo_x[x] = max(0, w.q[x].m0 - a.left);
-                hi_x[x] = min(a.T - 1, w.q[x].m0 + BM - 1 + a.right);
+                hi_x[x] = min(TT - 1, w.q[x].m0 + BM - 1 + a.right);
                 lo = min(lo, lo_x[x]);
                 hi = max(hi, hi_x[x]);
             }
@@ -435,10 +449,11 @@ __device__ __forceinline__ void softmax_tile(const TileCtx &k, const TcPrefillAr
 // (swa_prefill_chunk), compiled as its own kernel so that the other calls
 // keep 32-bit key positions, no ring branches and their four-map argument
 // list (two more tensor-map arguments alone cost those launches 2%).
-template <int D, bool RING, bool SINKS>
+template <int D, bool RING, bool SINKS, bool VARLEN>
 __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                                             const CUtensorMap *tmO, const CUtensorMap *tmKr, const CUtensorMap *tmVr,
-                                            const TcPrefillArgs &a, const RingArgs &ring, const int n_mode1)
+                                            const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl,
+                                            const int n_mode1)
 {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -450,7 +465,16 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const Work w = make_work<RING, SINKS>(a, ring, n_mode1);
+    const Work w = make_work<RING, SINKS, VARLEN>(a, ring, vl, n_mode1);
+    if constexpr (VARLEN) {
+        const int c0 = vl.cu[w.b], c1 = vl.cu[w.b + 1];
+        if ((c0 < 0 || c1 < c0 || c1 > a.T || c1 - c0 > vl.max_len) && threadIdx.x == 0)
+            atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+    }
+    // a packed-sequence unit past its sequence's end has nothing to do
+    if (VARLEN && !w.q[0].active) return;
+    const int tb = VARLEN ? 0 : w.b;         // batch coordinate of the tensors
+    const int trow0 = VARLEN ? vl.cu[w.b] : 0; // row of query/key position 0
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -501,7 +525,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                     if (w.q[x].active)
                         for (int ch = 0; ch < C::NCH; ++ch)
                             tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, tmQ, &bars->q_full, ch * C::E, w.q[x].h,
-                                        w.q[x].m0, w.b);
+                                        w.q[x].m0 + trow0, tb);
             }
         } else {
             for (int x = 0; x < 2; ++x)
@@ -586,7 +610,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                         mbar_expect_tx(&bars->k_full[st], C::KTILE);
                         for (int ch = 0; ch < C::NCH; ++ch)
                             tma_load_4d(sK + st * C::KTILE + ch * C::KCH, tmK, &bars->k_full[st], ch * C::E, w.hk,
-                                        key0, w.b);
+                                        key0 + trow0, tb);
                     }
                 } else {
                     if constexpr (SINKS)
@@ -607,7 +631,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                         mbar_expect_tx(&bars->v_full[st], C::KTILE);
                         for (int ch = 0; ch < C::NCH; ++ch)
                             tma_load_4d(sV + st * C::KTILE + ch * C::KCH, tmV, &bars->v_full[st], ch * C::E, w.hk,
-                                        key0, w.b);
+                                        key0 + trow0, tb);
                     }
                 } else {
                     if constexpr (SINKS)
@@ -726,7 +750,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
         // key positions: 64-bit only for a chunk continuing a ring
         typedef typename std::conditional<RING, long long, int>::type kpos_t;
         const long long p0 = RING ? w.p0 : 0;
-#define KEND (RING ? (kpos_t)w.kend : (kpos_t)a.T) // one past the last key
+#define KEND ((RING || VARLEN) ? (kpos_t)w.kend : (kpos_t)a.T) // one past the last key
         long long i_row;                        // absolute query position
         if (w.mode == 0) i_row = p0 + qt.m0 + r;
         else i_row = (qt.active && r < qt.nrows) ? gb[qt.gt * BM + r] : 0;
@@ -819,14 +843,17 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
             const int cl = nx - 1;
             ok = warp_wait_bounded(&bars->pv_done[x][cl & 1], (cl >> 1) & 1, ctl);
         }
-        const bool direct = (w.mode == 1) || (a.gidx != nullptr && a.g > 0);
+        // rows written one by one: dense global rows, band rows next to global
+        // ones, and the last tile of a packed sequence (a tile store would
+        // run into the next sequence)
+        const bool direct = (w.mode == 1) || (a.gidx != nullptr && a.g > 0) || (VARLEN && qt.nrows < BM);
         uint8_t *stage = sQ + x * C::QTILE;
         if (ok && qt.active) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o);
             bool skip_row = !row_real;
-            if (w.mode == 0 && direct && row_real) {
+            if (!VARLEN && w.mode == 0 && direct && row_real) {
                 // rows of global tokens are written by the dense-row CTAs
                 int lo = 0, hi = a.g;
                 while (lo < hi) {
@@ -851,7 +878,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                     const int e = cc * 16 + u * 8;
                     if (direct) {
                         if (!skip_row) {
-                            __nv_bfloat16 *dst = o + (((long long)w.b * a.T + i_out) * a.Hq + qt.h) * D + e;
+                            __nv_bfloat16 *dst = o + (((long long)tb * a.T + trow0 + i_out) * a.Hq + qt.h) * D + e;
                             *reinterpret_cast<uint4 *>(dst) = pk;
                         }
                     } else {
@@ -860,7 +887,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                 }
             }
             if (a.lse && row_real && !skip_row)
-                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_out] =
+                a.lse[((long long)tb * a.Hq + qt.h) * a.T + trow0 + i_out] =
                     (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
         // staging tile complete -> one thread per warpgroup stores it
@@ -871,7 +898,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
             if (lane == 0) mbar_arrive(&bars->epi[x]);
             if (r == 0 && wait_bounded(&bars->epi[x], 0, ctl) && !bars->abort) {
                 for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_store_4d(tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
+                    tma_store_4d(tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0 + trow0, tb);
                 tma_store_commit();
                 tma_store_wait_all();
             }
@@ -892,7 +919,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                           const TcPrefillArgs a, const int n_mode1)
 {
-    prefill_cta<D, false, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
+    prefill_cta<D, false, false, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, VarlenArgs{}, n_mode1);
 }
 
 // Causal window plus attention sinks (a.gidx null, a.g sinks): the sink keys
@@ -903,7 +930,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                              const TcPrefillArgs a, const int n_mode1)
 {
-    prefill_cta<D, false, true>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, n_mode1);
+    prefill_cta<D, false, true, false>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, VarlenArgs{}, n_mode1);
+}
+
+// Packed variable-length sequences: [total,H,d] tensors, sequence b in rows
+// cu[b] .. cu[b+1]-1.
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    swa_prefill_varlen_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                              const TcPrefillArgs a, const VarlenArgs vl, const int n_mode1)
+{
+    prefill_cta<D, false, false, true>(&tmQ, &tmK, &tmV, &tmO, nullptr, nullptr, a, RingArgs{}, vl, n_mode1);
 }
 
 template <int D>
@@ -913,7 +951,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
                             const TcPrefillArgs a, const RingArgs ring, const int n_mode1)
 {
-    prefill_cta<D, true, false>(&tmQ, &tmK, &tmV, &tmO, &tmKr, &tmVr, a, ring, n_mode1);
+    prefill_cta<D, true, false, false>(&tmQ, &tmK, &tmV, &tmO, &tmKr, &tmVr, a, ring, VarlenArgs{}, n_mode1);
 }
 
 // ------------------------------------------------------------------ host --
@@ -1032,12 +1070,52 @@ cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cu
 }
 
 template <int D>
+cudaError_t launch_varlen_d(const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s)
+{
+    using C = Cfg<D>;
+    // the packed tensors as one sequence of `total` rows
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map<D>(&mq, a.q, 1, a.T, a.Hq, BM) || !make_map<D>(&mk, a.k, 1, a.T, a.Hkv, BN) ||
+        !make_map<D>(&mv, a.v, 1, a.T, a.Hkv, BN) || !make_map<D>(&mo, a.o, 1, a.T, a.Hq, BM))
+        return cudaErrorInvalidValue;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(swa_prefill_varlen_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int G = a.Hq / a.Hkv;
+    const bool pair_heads = (G % 2) == 0;
+    const int nqt = (vl.max_len + BM - 1) / BM;
+    // units over (sequence, query tile [pair], head [pair]); those past a
+    // sequence's end return at once
+    const long long units = (long long)a.B * (pair_heads ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
+    if (units == 0) return cudaSuccess;
+    if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    swa_prefill_varlen_kernel<D><<<(int)units, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, vl, 0);
+    return cudaGetLastError();
+}
+
+template <int D>
 cudaError_t launch_d(int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     return ring.pos ? launch_dr<D, true>(mode, a, ring, s) : launch_dr<D, false>(mode, a, ring, s);
 }
 
 }  // namespace
+
+cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s)
+{
+    switch (d) {
+    case 32: return launch_varlen_d<32>(a, vl, s);
+    case 64: return launch_varlen_d<64>(a, vl, s);
+    case 128: return launch_varlen_d<128>(a, vl, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 // mode 0: band tiles (+ dense global-row CTAs first in the same grid when
 // global tokens are present); mode 1: dense global rows only.

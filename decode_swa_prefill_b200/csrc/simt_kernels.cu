@@ -149,8 +149,21 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
         for (long long j = 0; j < a.T; ++j) visit(j);
     } else {
         const long long ip = p0 + i;  // absolute position of the row
-        const long long lo = max(0LL, ip - a.left);
-        const long long hi = min(p0 + a.T - 1, ip + a.right);
+        long long first = 0, last = p0 + a.T - 1;  // the row's sequence
+        if (a.cu) {
+            // packed sequences: the one holding row i (kept inside the rows
+            // even for an inconsistent cu)
+            int s0 = 0, s1 = a.nseq;
+            while (s1 - s0 > 1) {
+                const int mid = (s0 + s1) / 2;
+                if (a.cu[mid] <= i) s0 = mid;
+                else s1 = mid;
+            }
+            first = max(0LL, (long long)a.cu[s0]);
+            last = min((long long)a.T - 1, (long long)a.cu[s0 + 1] - 1);
+        }
+        const long long lo = max(first, ip - a.left);
+        const long long hi = min(last, ip + a.right);
         if (!gb && a.g > 0)  // sinks older than the window
             for (long long j = 0; j < min((long long)a.g, lo); ++j) visit(j);
         for (long long j = lo; j <= hi; ++j) visit(j);

@@ -239,6 +239,35 @@ swa_status swa_prefill_dilated(const void *q, const void *k, const void *v, void
     return SWA_OK;
 }
 
+swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int32_t *cu_seqlens, int nseq, int total, int max_seqlen, int Hq, int Hkv, int d,
+                              int W, float scale, swa_dtype dt, void *stream)
+{
+    swa_status st = check_prefill(q, k, v, o, lse, 1, total, Hq, Hkv, d, W, scale, dt);
+    if (st != SWA_OK) return st;
+    if (nseq < 0 || max_seqlen < 0 || max_seqlen > total) return SWA_ERR_INVALID_ARG;
+    if (nseq == 0 || total == 0 || max_seqlen == 0) return SWA_OK;
+    if (!cu_seqlens || !aligned(cu_seqlens, 4)) return SWA_ERR_INVALID_ARG;
+    const int left = W - 1 < max_seqlen ? W - 1 : max_seqlen;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dt == SWA_DTYPE_F32) {
+        swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<float *>(o), lse, 1, total, Hq, Hkv, d, left, 0,
+                              nullptr, 0, scale};
+        a.cu = cu_seqlens;
+        a.nseq = nseq;
+        return from_cuda(swa::launch_prefill_f32(a, s));
+    }
+    swa::TcPrefillArgs a{};
+    a.B = nseq; a.T = total; a.Hq = Hq; a.Hkv = Hkv;
+    a.left = left; a.right = 0;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.lse = lse; a.gidx = nullptr; a.g = 0;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    if ((st = ctl(&a.ctl)) != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_varlen(d, a, swa::VarlenArgs{cu_seqlens, max_seqlen}, s));
+}
+
 swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink, int B,
                              int T, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
 {

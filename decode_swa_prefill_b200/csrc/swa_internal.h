@@ -52,6 +52,15 @@ struct RingArgs {
 // mode 1: one CTA per (128 global rows, head, batch): dense rows over all keys
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s);
 
+// Packed variable-length sequences (causal band mode): q/k/v/o are
+// [total,H,d] (TcPrefillArgs.T = total, B = number of sequences) and
+// sequence b holds rows cu[b] .. cu[b+1]-1, none longer than max_len.
+struct VarlenArgs {
+    const int32_t *cu;        // device [B+1]
+    int max_len;
+};
+cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s);
+
 // ---- SIMT kernels ----
 // Attention sinks in the prefill calls: gidx == null with g > 0 means the
 // first g positions of each sequence are keys every later query sees
@@ -69,6 +78,10 @@ struct F32PrefillArgs {
     const float *kc, *vc;
     int W_ring;
     DeviceCtl ctl;
+    // packed sequences (B == 1, T = total rows): sequence s holds rows
+    // cu[s] .. cu[s+1]-1 (null: one sequence per batch row)
+    const int32_t *cu;
+    int nseq;
 };
 cudaError_t launch_prefill_f32(const F32PrefillArgs &a, cudaStream_t s);
 

@@ -88,6 +88,23 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
                               swa_dtype dt, void *stream);
 
 /*
+ * Causal sliding-window prefill over packed sequences of different lengths
+ * (variable-length batches): every sequence is its own causal prefill
+ * (robocikowo.com opening definition); no row sees another sequence.
+ *   q, o : [total,Hq,d]   k, v : [total,Hkv,d]   (rows of all sequences, one
+ *          after the other)
+ *   cu_seqlens : device int32 [nseq+1]: sequence s holds rows cu[s] ..
+ *          cu[s+1]-1; cu[0] = 0, non-decreasing, cu[nseq] = total, each
+ *          length <= max_seqlen (an entry breaking this makes its sequence
+ *          empty and records SWA_ERR_INVALID_ARG in the device status word)
+ *   lse  : nullable fp32 [Hq,total]
+ *   0 <= max_seqlen <= total; other arguments as swa_prefill.
+ */
+swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int32_t *cu_seqlens, int nseq, int total, int max_seqlen,
+                              int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream);
+
+/*
  * Dilated sliding-window prefill (aivaro.ru section 4.2: instead of all
  * neighbours, every dil-th token, which widens the span without more keys).
  *   symmetric = 0: query i sees keys i - dil*m, m = 0 .. W-1 (j >= 0)

@@ -127,6 +127,19 @@ def test_dilated_rejects(lib):
     assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 1      # workspace needs 256-byte alignment
 
 
+def test_varlen_rejects(lib):
+    f = lib.swa_prefill_varlen
+    call = lambda cu=FAKE, nseq=3, total=300, maxl=128, d=64: f(FAKE, FAKE, FAKE, FAKE, NULL, cu, nseq, total, maxl,
+                                                                8, 2, d, 64, 0.125, 1, NULL)
+    assert call(cu=NULL) == 1
+    assert call(cu=ctypes.c_void_p((1 << 20) + 2)) == 1
+    assert call(nseq=-1) == 1
+    assert call(maxl=301) == 1
+    assert call(d=48) == 2
+    assert call(nseq=0, cu=NULL) == 0
+    assert f(NULL, NULL, NULL, NULL, NULL, NULL, 2, 0, 0, 8, 2, 64, 64, 0.125, 1, NULL) == 0   # no rows
+
+
 def test_append_rejects(lib):
     f = lib.swa_cache_append
     assert f(FAKE, FAKE, FAKE, FAKE, NULL, NULL, 2, 1, 8, 128, 64, 1, NULL) == 1      # no pos
