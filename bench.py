@@ -22,6 +22,7 @@ collective on the data path); ranks are timed on the device and the slowest
 rank's time is reported.
 """
 import argparse
+import itertools
 import hashlib
 import json
 import os
@@ -294,6 +295,7 @@ def gpu_arm(args, world, rank, local):
     chunk = chunk_arm(swa, dev, args)
     sinks = sinks_arm(swa, dev, args, load_peaks()[0])
     dilated = dilated_arm(swa, dev, args, load_peaks()[0])
+    varlen = varlen_arm(swa, dev, args, load_peaks()[0])
 
     peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
@@ -325,6 +327,7 @@ def gpu_arm(args, world, rank, local):
             "chunk_prefill": chunk,
             "sinks": sinks,
             "dilated": dilated,
+            "varlen": varlen,
             "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
@@ -438,6 +441,30 @@ def dilated_arm(swa, dev, args, peaks):
     tf = flops / (ms * 1e-3) / 1e12
     return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "flops": flops, "dil": dil, "workload": "longformer_B8_T4096_h12_d64_W512_dil2_symmetric"}
+
+
+def varlen_arm(swa, dev, args, peaks):
+    """Packed variable-length prefill: 8 sequences of seeded lengths summing
+    to 32768 tokens, Mistral-7B heads and window: not part of the step."""
+    w = wl.MISTRAL_PREFILL
+    lengths = wl.varlen_lengths(8, w.T, seed=6)
+    q, k, v = (t[0].to(dev) for t in wl.prefill_inputs(1, w.T, w.Hq, w.Hkv, w.d, w.dtype, w.seed))
+    cu = torch.tensor([0] + list(itertools.accumulate(lengths)), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    flops = sum(causal_pairs(n, w.W) for n in lengths) * w.Hq * 4 * w.d
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill_varlen(q, k, v, cu, w.W, max_seqlen=max(lengths), o=o)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "flops": flops, "lengths": lengths}
 
 
 def sink_pairs(T, W, s):

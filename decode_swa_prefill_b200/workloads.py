@@ -59,6 +59,15 @@ MISTRAL_CHUNK = Workload("mistral7b_chunk_B4_n4096_h32x8_d128_W4096", "prefill_c
 ALL = [TOY, TINYMISTRAL, MISTRAL_PREFILL, MISTRAL_DECODE, LONGFORMER, MISTRAL_CHUNK]
 
 
+def varlen_lengths(n, total, seed, min_len=1):
+    """n sequence lengths summing to `total`, drawn from a seeded uniform
+    split (each at least min_len)."""
+    g = _gen(seed + 3000)
+    cuts = torch.sort(torch.randperm(total - n * min_len + n - 1, generator=g)[:n - 1]).values
+    edges = torch.cat([torch.tensor([-1]), cuts, torch.tensor([total - n * min_len + n - 1])])
+    return [int(x) - 1 + min_len for x in (edges[1:] - edges[:-1])]
+
+
 def _gen(seed: int) -> torch.Generator:
     return torch.Generator().manual_seed(seed)
 
