@@ -446,12 +446,16 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
-    auto krow = [&](int sl) -> const __nv_bfloat16 * {
-        if (SINKS && sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
+    // row sources: the ring, or (the last split of a call with sinks) the
+    // ring and then the sink caches
+    auto ring_k = [&](int sl) -> const __nv_bfloat16 * { return kb + (long long)sl * D; };
+    auto ring_v = [&](int sl) -> const __nv_bfloat16 * { return vb + (long long)sl * D; };
+    auto tail_k = [&](int sl) -> const __nv_bfloat16 * {
+        if (sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
         return kb + (long long)sl * D;
     };
-    auto vrow = [&](int sl) -> const __nv_bfloat16 * {
-        if (SINKS && sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.vs) + sink0 + (long long)(sl - n_valid) * D;
+    auto tail_v = [&](int sl) -> const __nv_bfloat16 * {
+        if (sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.vs) + sink0 + (long long)(sl - n_valid) * D;
         return vb + (long long)sl * D;
     };
 
@@ -468,6 +472,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
         for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
     }
 
+    auto run = [&](auto krow, auto vrow) {
     for (int base = s_begin + warp * BATCH; base < s_end; base += DEC_WARPS * BATCH) {
         uint4 kr[NBL], vr[NBL];
 #pragma unroll
@@ -543,6 +548,13 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
                 acc[g][3] = fma2(p2, v3, acc[g][3]);
             }
         }
+    }
+    };
+    if constexpr (SINKS) {
+        if (split == a.splits - 1) run(tail_k, tail_v);
+        else run(ring_k, ring_v);
+    } else {
+        run(ring_k, ring_v);
     }
     // sum the row groups' accumulators (same softmax reference per head)
 #pragma unroll
