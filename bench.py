@@ -520,40 +520,71 @@ def e2e_arm(st, args, world, dev, step_flops):
     """Per step: pinned host -> device copies of the step's inputs, the four
     calls, device -> host copies of the outputs.  The decode ring is resident
     model state (like weights); the new token's k/v, q and positions are
-    inputs."""
+    inputs.  Steps are pipelined over three streams and two device buffer
+    sets: step i+1's inputs are copied in and step i-1's outputs copied out
+    while step i computes, each step waiting for exactly the copies it
+    needs."""
+    import copy
+
     hp, hl, hd = st.host["prefill"], st.host["lf"], st.host["dec"]
-    ins = [(hp["q"], st.q), (hp["k"], st.k), (hp["v"], st.v), (hl["q"], st.lq), (hl["k"], st.lk),
-           (hl["v"], st.lv), (hl["global_idx"], st.lg), (hd["q"], st.dq), (hd["k_new"], st.kn),
-           (hd["v_new"], st.vn), (hd["pos"], st.pos)]
-    ins = [(h.pin_memory(), d) for h, d in ins]
-    outs = [(st.o, torch.empty(st.o.shape, dtype=st.o.dtype, pin_memory=True)),
-            (st.lo, torch.empty(st.lo.shape, dtype=st.lo.dtype, pin_memory=True)),
-            (st.do, torch.empty(st.do.shape, dtype=st.do.dtype, pin_memory=True))]
-    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
-    d2h = sum(h.numel() * h.element_size() for _, h in outs)
-    steps = max(3, args.steps // 4)
+    in_names = ["q", "k", "v", "lq", "lk", "lv", "lg", "dq", "kn", "vn", "pos"]
+    out_names = ["o", "lo", "do"]
+    host_in = [hp["q"], hp["k"], hp["v"], hl["q"], hl["k"], hl["v"], hl["global_idx"], hd["q"], hd["k_new"],
+               hd["v_new"], hd["pos"]]
+    host_in = [h.pin_memory() for h in host_in]
+    host_out = [torch.empty(getattr(st, n).shape, dtype=getattr(st, n).dtype, pin_memory=True) for n in out_names]
+    # a second set of per-step buffers; the ring and the decode workspace are shared
+    alt = copy.copy(st)
+    for n in in_names + out_names:
+        setattr(alt, n, torch.empty_like(getattr(st, n)))
+    sets = [st, alt]
+    h2d = sum(h.numel() * h.element_size() for h in host_in)
+    d2h = sum(h.numel() * h.element_size() for h in host_out)
+    steps = max(4, args.steps // 4)
+    s_in, s_cp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def one():
-        for h, d in ins:
-            d.copy_(h, non_blocking=True)
-        st.run()
-        for d, h in outs:
-            h.copy_(d, non_blocking=True)
+    def pipeline(n):
+        ev = {k: [torch.cuda.Event() for _ in range(n)] for k in ("in", "cp", "out")}
+        for i in range(n):
+            bs = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev["cp"][i - 2])      # set no longer read by compute i-2
+                for h, name in zip(host_in, in_names):
+                    getattr(bs, name).copy_(h, non_blocking=True)
+                ev["in"][i].record(s_in)
+            with torch.cuda.stream(s_cp):
+                s_cp.wait_event(ev["in"][i])
+                if i >= 2:
+                    s_cp.wait_event(ev["out"][i - 2])     # outputs of step i-2 copied out
+                bs.run()
+                ev["cp"][i].record(s_cp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["cp"][i])
+                for name, h in zip(out_names, host_out):
+                    h.copy_(getattr(bs, name), non_blocking=True)
+                ev["out"][i].record(s_out)
+        return ev
 
-    one()
+    pipeline(2)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     a.record()
-    for _ in range(steps):
-        one()
+    for s_ in (s_in, s_cp, s_out):
+        s_.wait_event(a)
+    ev = pipeline(steps)
+    cur = torch.cuda.current_stream()
+    for k in ("in", "cp", "out"):
+        cur.wait_event(ev[k][-1])
     b.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world) / steps
     return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 3), "steps": steps,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "copies": "pipelined: inputs of step i+1 and outputs of step i-1 move while step i computes"}
 
 
 # ------------------------------------------------------- oracle (CPU) --
