@@ -100,11 +100,6 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes)
 {
@@ -255,13 +250,6 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t *r)
-{
-    tmem_st32(taddr, reinterpret_cast<const float *>(r));
-}
-
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 // Wait for this thread's TMEM loads and tie the 16 registers of `v` to the
 // wait, so no use of them can be scheduled before the data has arrived.
 __device__ __forceinline__ void tmem_ld_wait_dep16(float *v)
@@ -332,19 +320,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, i
            | (static_cast<uint32_t>(b_mn) << 16)       // B major
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
-}
-
-// Warpgroup register reallocation (all 128 threads of the warpgroup).
-template <int N>
-__device__ __forceinline__ void reg_alloc()
-{
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-template <int N>
-__device__ __forceinline__ void reg_dealloc()
-{
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------ numerics --
