@@ -92,8 +92,9 @@ def load_peaks():
 
 # the sources each recorded kernel is built from
 KERNEL_SOURCES = {
-    "prefill_mistral": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h"),
-    "longformer": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h"),
+    "prefill_mistral": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
+    "longformer": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
+    "tinymistral": ("narrow_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
     "decode_mistral": ("simt_kernels.cu", "ptx.cuh", "swa_internal.h"),
 }
 

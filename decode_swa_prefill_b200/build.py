@@ -11,8 +11,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libswa.so")
-SOURCES = ["swa_abi.cu", "prefill_tc.cu", "simt_kernels.cu", "decode_noalloc.cu", "dilated.cu"]
-HEADERS = ["ptx.cuh", "swa_internal.h"]
+SOURCES = ["swa_abi.cu", "prefill_tc.cu", "narrow_tc.cu", "simt_kernels.cu", "decode_noalloc.cu", "dilated.cu"]
+HEADERS = ["ptx.cuh", "swa_internal.h", "tma_map.h"]
 
 
 def nvcc():

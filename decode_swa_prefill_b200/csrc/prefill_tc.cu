@@ -56,6 +56,7 @@
 
 #include "ptx.cuh"
 #include "swa_internal.h"
+#include "tma_map.h"
 
 namespace swa {
 namespace {
@@ -956,40 +957,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 // ------------------------------------------------------------------ host --
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // [B,T,H,D] bf16 viewed as a 4-D tensor (D, H, T, B); box = one chunk of
 // `rows` rows of one head.
 template <int D>
 bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int rows)
 {
-    using C = Cfg<D>;
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    cuuint32_t box[4] = {(cuuint32_t)C::E, 1, (cuuint32_t)rows, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     C::RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return make_bthd_map(m, ptr, B, T, H, D, rows);
 }
 
 // Ring cache [B,Hkv,W,D] bf16 viewed as (D, W, Hkv, B); box = one chunk of
@@ -1118,9 +1091,12 @@ cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArg
 }
 
 // mode 0: band tiles (+ dense global-row CTAs first in the same grid when
-// global tokens are present); mode 1: dense global rows only.
+// global tokens are present), or the narrow-window kernel; mode 1: dense
+// global rows only.
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
+    // a causal window of at most 64 keys: the single-pass kernel
+    if (mode == 0 && ring.pos == nullptr && prefill_narrow_applies(d, a)) return launch_prefill_narrow(d, a, s);
     switch (d) {
     case 32: return launch_d<32>(mode, a, ring, s);
     case 64: return launch_d<64>(mode, a, ring, s);

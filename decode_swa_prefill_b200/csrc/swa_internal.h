@@ -52,6 +52,12 @@ struct RingArgs {
 // mode 1: one CTA per (128 global rows, head, batch): dense rows over all keys
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s);
 
+// Causal window of at most 64 keys (left <= 63, right 0, no global keys or
+// sinks), d = 32 or 64: persistent single-pass kernel whose S tile holds
+// every key a 128-row query tile sees.
+bool prefill_narrow_applies(int d, const TcPrefillArgs &a);
+cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s);
+
 // Packed variable-length sequences (causal band mode): q/k/v/o are
 // [total,H,d] (TcPrefillArgs.T = total, B = number of sequences) and
 // sequence b holds rows cu[b] .. cu[b+1]-1, none longer than max_len.
