@@ -375,7 +375,8 @@ def tinymistral_arm(swa, dev, args):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
             "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "bytes": nbytes, "flops": flops,
-            "l2": "flushed before each launch"}
+            "l2": "flushed before each launch", "kernel": "swa_prefill_narrow_kernel",
+            "traffic": recorded_traffic("tinymistral")}
 
 
 def chunk_pairs(n, W, p0):

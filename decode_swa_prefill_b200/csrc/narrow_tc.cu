@@ -7,12 +7,13 @@
 // per-tile pipeline fill and drain dominate.  A tile at rows q0 .. q0+127
 // sees keys q0-PAD .. q0+127 at most (PAD = 32 for W <= 32, 64 for W <= 64),
 // so one S = Q K^T of N = 128+PAD columns holds every score of the tile and
-// the softmax is a single pass: no running maximum, no rescaling of O, P
-// normalised by its row sum before the PV product, O final when PV is done.
+// the softmax is a single pass: one row maximum, no rescaling of O, and O
+// divided by the row sum in the epilogue once the PV product is done.
 //
 // Persistent CTAs, one per SM (two TMEM buffers take all 512 columns), walk
-// units of (batch, kv head, query tile) with a stride of the grid size; the
-// G query heads of a unit share its K/V tile and are its jobs.  Job j uses
+// units of (batch, kv head, query tile[, slice of the query heads]) with a
+// stride of the grid size; the query heads of a unit share its K/V tile and
+// are its jobs.  Job j uses
 // TMEM buffer j & 1:
 //   O[b]  columns 256b .. 256b+d-1       fp32 output of the job
 //   S[b]  columns 256b+64 .. +128+PAD-1  fp32 scores; P (bf16 pairs) over
@@ -24,9 +25,12 @@
 //              (128 rows) per job into rings of 2 and 4 stages
 //   warp 9     TMEM allocator and MMA issuer (lane 0): QK^T of job j, then
 //              PV of job j-1, so a QK^T runs while the previous job's
-//              softmax works
+//              softmax works.  S[b] is rewritten once the PV that read P[b]
+//              has completed, O[b] once the epilogue two jobs back has read
+//              it: the epilogue is off the MMA's critical path.
 // A warp only computes the 32-key chunks its rows can see (two for PAD 32,
-// three for PAD 64) and writes zeros to the rest of its P columns.
+// three for PAD 64) and writes zeros to the rest of its P columns.  The
+// softmax is issue-bound, so every exponential runs on the MUFU.
 //
 // Every mbarrier wait is bounded: on expiry the CTA records
 // SWA_STATUS_TIMEOUT, drains its in-flight copies and MMAs with a second
@@ -43,30 +47,39 @@ namespace swa {
 namespace {
 
 constexpr int NB_BM = 128;          // query rows per tile (= TMEM lanes)
-constexpr int NB_QST = 4;           // Q stages
-constexpr int NB_KVST = 2;          // K/V stages
+constexpr int NB_QST_MAX = 8;      // Q stages (at most)
+constexpr int NB_KVST_MAX = 4;     // K/V stages (at most)
 constexpr int NB_THREADS = 320;
-constexpr int NB_POLY_EVERY = 4;    // every 4th pair of exponentials on the FMA pipe
 
-template <int D, int PAD>
+// HP heads side by side per tile row: HP = 2 for d = 32 loads two adjacent
+// heads as one 128-byte row (one TMA row request instead of two; rows of 64
+// bytes halve what a load moves per request), and the MMAs of head x of the
+// pair start 64 bytes into the row.
+template <int D, int PAD, int HP>
 struct NCfg {
     static constexpr int KEYS = NB_BM + PAD;                 // key rows of a unit
-    static constexpr int RB = (D * 2 >= 128) ? 128 : D * 2;  // bytes per swizzled row
-    static constexpr int QTILE = NB_BM * D * 2;
-    static constexpr int KVTILE = KEYS * D * 2;
+    static constexpr int RD = HP * D;                        // elements per tile row
+    static constexpr int RB = (RD * 2 >= 128) ? 128 : RD * 2; // bytes per swizzled row
+    static constexpr int QTILE = NB_BM * RD * 2;             // HP jobs' Q
+    static constexpr int KVTILE = KEYS * RD * 2;             // HP kv heads' K (or V)
     static constexpr uint32_t LAYOUT = (RB == 128) ? UMMA_SW128 : UMMA_SW64;
     static constexpr int NCHK = PAD / 32 + 1;                // live 32-key chunks per warp
+    // prefetch depth: a load takes a few microseconds, several units' worth
+    // of jobs, so as many stages as shared memory holds
+    static constexpr int QST = RD == 32 ? 8 : 4;
+    static constexpr int KVST = RD == 32 ? 4 : 3;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + NB_QST * QTILE;
-    static constexpr int OFF_V = OFF_K + NB_KVST * KVTILE;
-    static constexpr int OFF_BAR = OFF_V + NB_KVST * KVTILE;
+    static constexpr int OFF_K = OFF_Q + QST * QTILE;
+    static constexpr int OFF_V = OFF_K + KVST * KVTILE;
+    static constexpr int OFF_BAR = OFF_V + KVST * KVTILE;
     // + room to align the base to 1 KiB; more than half the SM's shared
     // memory, so that a second CTA (which would wait for TMEM) never shares
     // the SM
     static constexpr int SMEM_NEED = OFF_BAR + 256 + 1024;
     static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
     static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(D == 32 || D == 64, "head dim: one swizzle chunk per row");
+    static_assert(RD == 32 || RD == 64, "one swizzle chunk per tile row");
+    static_assert(HP == 1 || HP == 2, "heads per row");
     static_assert(PAD == 32 || PAD == 64, "pad");
     static_assert(64 + KEYS <= 256 && D <= 64, "one TMEM buffer = 256 columns");
     static_assert(QTILE % 1024 == 0 && KVTILE % 1024 == 0, "1 KiB aligned stages");
@@ -78,10 +91,10 @@ __host__ __device__ constexpr uint32_t nb_col_o(int b) { return 256u * b; }
 __host__ __device__ constexpr uint32_t nb_col_s(int b) { return 256u * b + 64u; }
 
 struct NBars {
-    uint64_t q_full[NB_QST];
-    uint64_t q_empty[NB_QST];
-    uint64_t kv_full[NB_KVST];
-    uint64_t kv_empty[NB_KVST];
+    uint64_t q_full[NB_QST_MAX];
+    uint64_t q_empty[NB_QST_MAX];
+    uint64_t kv_full[NB_KVST_MAX];
+    uint64_t kv_empty[NB_KVST_MAX];
     uint64_t s_full[2];
     uint64_t p_full[2];     // one arrival per softmax warp
     uint64_t o_full[2];
@@ -99,28 +112,32 @@ __device__ __forceinline__ void nb_drain_wait(uint64_t *bar, uint32_t parity, un
     }
 }
 
-// Unit u -> (batch, kv head, query tile); consecutive units are consecutive
-// query tiles of one (batch, kv head), so neighbouring CTAs share K/V rows in
-// L2.
+// Unit u -> (batch, group of HP kv heads, query tile, slice of the group's
+// query heads); consecutive units share K/V rows (the slices of one tile,
+// then the next tile), so neighbouring CTAs find them in L2.
 struct NUnit {
-    int b, hk, q0;
+    int b, kp, q0, h0; // kp: kv head group (tile row index); h0: first query head
 };
-__device__ __forceinline__ NUnit nb_unit(int u, int Hkv, int nqt)
+__device__ __forceinline__ NUnit nb_unit(int u, int n_kp, int nqt, int n_slice, int gs)
 {
     NUnit x;
+    x.h0 = (u % n_slice) * gs;
+    u /= n_slice;
     x.q0 = (u % nqt) * NB_BM;
     const int r = u / nqt;
-    x.hk = r % Hkv;
-    x.b = r / Hkv;
+    x.kp = r % n_kp;
+    x.b = r / n_kp;
+    x.h0 += x.kp * gs * n_slice;
     return x;
 }
 
-template <int D, int PAD>
+template <int D, int PAD, int HP>
 __global__ void __launch_bounds__(NB_THREADS, 1)
     swa_prefill_narrow_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                              const __grid_constant__ CUtensorMap tmV, const TcPrefillArgs a, const int n_units)
+                              const __grid_constant__ CUtensorMap tmV, const TcPrefillArgs a, const int n_units,
+                              const int n_slice)
 {
-    using C = NCfg<D, PAD>;
+    using C = NCfg<D, PAD, HP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + C::OFF_Q;
@@ -130,16 +147,18 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int G = a.Hq / a.Hkv;
+    const int Gq = a.Hq / a.Hkv;             // query heads per kv head
+    const int G = HP * Gq / n_slice;         // jobs (query heads) per unit, a multiple of HP
+    const int n_kp = a.Hkv / HP;
     const int nqt = (a.T + NB_BM - 1) / NB_BM;
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NB_QST; ++s) {
+        for (int s = 0; s < C::QST; ++s) {
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
         }
-        for (int s = 0; s < NB_KVST; ++s) {
+        for (int s = 0; s < C::KVST; ++s) {
             mbar_init(&bars->kv_full[s], 1);
             mbar_init(&bars->kv_empty[s], 1);
         }
@@ -166,37 +185,38 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------ producer --
-        int qiss[NB_QST] = {}, kviss[NB_KVST] = {};
+        int qiss[C::QST] = {}, kviss[C::KVST] = {};
         bool ok = true;
         int jq = 0, it = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-            const NUnit x = nb_unit(u, a.Hkv, nqt);
-            const int ks = it % NB_KVST;
-            ok = warp_wait_bounded(&bars->kv_empty[ks], ((it / NB_KVST) & 1) ^ 1, ctl);
+            const NUnit x = nb_unit(u, n_kp, nqt, n_slice, G);
+            const int ks = it % C::KVST;
+            ok = warp_wait_bounded(&bars->kv_empty[ks], ((it / C::KVST) & 1) ^ 1, ctl);
             if (!ok) break;
             if (lane == 0) {
                 // rows q0-PAD .. q0+127; rows before 0 or past T read zeros
                 mbar_expect_tx(&bars->kv_full[ks], 2 * C::KVTILE);
-                tma_load_4d(sK + ks * C::KVTILE, &tmK, &bars->kv_full[ks], 0, x.hk, x.q0 - PAD, x.b);
-                tma_load_4d(sV + ks * C::KVTILE, &tmV, &bars->kv_full[ks], 0, x.hk, x.q0 - PAD, x.b);
+                tma_load_4d(sK + ks * C::KVTILE, &tmK, &bars->kv_full[ks], 0, x.kp, x.q0 - PAD, x.b);
+                tma_load_4d(sV + ks * C::KVTILE, &tmV, &bars->kv_full[ks], 0, x.kp, x.q0 - PAD, x.b);
             }
             kviss[ks]++;
-            for (int g = 0; g < G && ok; ++g, ++jq) {
-                const int qs = jq % NB_QST;
-                ok = warp_wait_bounded(&bars->q_empty[qs], ((jq / NB_QST) & 1) ^ 1, ctl);
+            // one Q tile per HP jobs (query heads h0+g .. h0+g+HP-1)
+            for (int g = 0; g < G && ok; g += HP, ++jq) {
+                const int qs = jq % C::QST;
+                ok = warp_wait_bounded(&bars->q_empty[qs], ((jq / C::QST) & 1) ^ 1, ctl);
                 if (!ok) break;
                 if (lane == 0) {
                     mbar_expect_tx(&bars->q_full[qs], C::QTILE);
-                    tma_load_4d(sQ + qs * C::QTILE, &tmQ, &bars->q_full[qs], 0, x.hk * G + g, x.q0, x.b);
+                    tma_load_4d(sQ + qs * C::QTILE, &tmQ, &bars->q_full[qs], 0, (x.h0 + g) / HP, x.q0, x.b);
                 }
                 qiss[qs]++;
             }
         }
         if (!ok && lane == 0) {
             // let our own copies land before the CTA's shared memory goes away
-            for (int s = 0; s < NB_QST; ++s)
+            for (int s = 0; s < C::QST; ++s)
                 if (qiss[s] > 0) nb_drain_wait(&bars->q_full[s], (qiss[s] - 1) & 1, a.ctl.limit_ns);
-            for (int s = 0; s < NB_KVST; ++s)
+            for (int s = 0; s < C::KVST; ++s)
                 if (kviss[s] > 0) nb_drain_wait(&bars->kv_full[s], (kviss[s] - 1) & 1, a.ctl.limit_ns);
         }
     } else if (warp == 9) {
@@ -210,14 +230,16 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
         const bool leader = lane == 0;
         bool ok = true;
         // the job whose PV is still to issue
-        int pj = -1, pks = 0;
+        int pj = -1, pks = 0, pkvo = 0;
         bool plast = false;
         auto pv_step = [&]() -> bool {
             const int b = pj & 1;
             if (!warp_wait_bounded(&bars->p_full[b], (pj >> 1) & 1, ctl)) return false;
+            // O[b] is free once job pj-2's epilogue has read it
+            if (pj >= 2 && !warp_wait_bounded(&bars->tmem_free[b], ((pj >> 1) - 1) & 1, ctl)) return false;
             tc_fence_after();
             if (leader) {
-                const uint64_t dv = dv0 + (uint64_t)((pks * C::KVTILE) >> 4);
+                const uint64_t dv = dv0 + (uint64_t)((pks * C::KVTILE + pkvo) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::KEYS / 16; ++kk)
                     mma_bf16_ts(tmem + nb_col_o(b), tmem + nb_col_s(b) + kk * 8,
@@ -231,31 +253,37 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
         };
         int j = 0, it = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
-            const int ks = it % NB_KVST;
+            const NUnit un = nb_unit(u, n_kp, nqt, n_slice, G);
+            const int ks = it % C::KVST;
             // the previous unit's last PV does not wait for this unit's K/V
             if (pj >= 0) ok = pv_step();
             if (!ok) break;
-            ok = warp_wait_bounded(&bars->kv_full[ks], (it / NB_KVST) & 1, ctl);
+            ok = warp_wait_bounded(&bars->kv_full[ks], (it / C::KVST) & 1, ctl);
             for (int g = 0; g < G && ok; ++g, ++j) {
-                const int qs = j % NB_QST, b = j & 1;
-                ok = warp_wait_bounded(&bars->q_full[qs], (j / NB_QST) & 1, ctl);
-                // S[b] / O[b] are free once job j-2's epilogue has read O[b]
-                if (ok && j >= 2) ok = warp_wait_bounded(&bars->tmem_free[b], ((j >> 1) - 1) & 1, ctl);
+                // Q tile of job pair j / HP; byte offsets of this job's head
+                // in the Q row and of its kv head in the K/V row
+                const int jp = j / HP, qs = jp % C::QST, b = j & 1;
+                const int h = un.h0 + g;
+                const int qo = (h % HP) * D * 2, kvo = ((h / Gq) % HP) * D * 2;
+                ok = warp_wait_bounded(&bars->q_full[qs], (jp / C::QST) & 1, ctl);
+                // S[b] (P of job j-2) is free once that job's PV has completed
+                if (ok && j >= 2) ok = warp_wait_bounded(&bars->o_full[b], ((j >> 1) - 1) & 1, ctl);
                 if (!ok) break;
                 tc_fence_after();
                 if (leader) {
-                    const uint64_t dq = dq0 + (uint64_t)((qs * C::QTILE) >> 4);
-                    const uint64_t dk = dk0 + (uint64_t)((ks * C::KVTILE) >> 4);
+                    const uint64_t dq = dq0 + (uint64_t)((qs * C::QTILE + qo) >> 4);
+                    const uint64_t dk = dk0 + (uint64_t)((ks * C::KVTILE + kvo) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
                         mma_bf16_ss(tmem + nb_col_s(b), dq + 2 * kk, dk + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
                     mma_commit(&bars->s_full[b]);
-                    mma_commit(&bars->q_empty[qs]);
+                    if (g % HP == HP - 1) mma_commit(&bars->q_empty[qs]);
                 }
                 __syncwarp();
                 if (pj >= 0) ok = pv_step();
                 pj = j;
                 pks = ks;
+                pkvo = kvo;
                 plast = (g == G - 1);
             }
         }
@@ -279,13 +307,15 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
         bool ok = true;
         int j = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            const NUnit un = nb_unit(u, a.Hkv, nqt);
+            const NUnit un = nb_unit(u, n_kp, nqt, n_slice, G);
             const int i = un.q0 + r;          // query position of this thread's row
             const bool row_real = i < a.T;
             // visible key columns of this row: key position q0-PAD+c for
-            // column c, from max(i-left, 0) to i
-            const int c_lo = max(r + PAD - a.left, PAD - un.q0);
-            const int c_hi = row_real ? r + PAD : -1;
+            // column c, from max(i-left, 0) to i; as offsets e from the
+            // warp's first live column 32*quarter: e_lo <= e <= lane + PAD
+            // (rows past T compute garbage that is never stored)
+            const int e_lo = max(r + PAD - a.left, PAD - un.q0) - quarter * 32;
+            const int e_hi = lane + PAD;
             for (int g = 0; g < G; ++g, ++j) {
                 if ((j & 1) != x) continue;
                 ok = warp_wait_bounded(&bars->s_full[x], (j >> 1) & 1, ctl);
@@ -297,36 +327,46 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
                 tmem_ld_wait_dep(sr);
 #pragma unroll
                 for (int cc = 1; cc < C::NCHK; ++cc) reg_fence32(sr + cc * 32);
-                float mx = -CUDART_INF_F;
+                // -inf outside the window: only the last chunk can pass e_hi
+                // (e_hi >= PAD), every chunk e_lo
 #pragma unroll
                 for (int e = 0; e < C::NCHK * 32; ++e) {
-                    const int c = quarter * 32 + e;
-                    if (c < c_lo || c > c_hi) sr[e] = -CUDART_INF_F;
-                    mx = fmaxf(mx, sr[e]);
+                    bool keep = e >= e_lo;
+                    if (e > PAD) keep = keep && e <= e_hi;
+                    sr[e] = keep ? sr[e] : -CUDART_INF_F;
                 }
+                float mx4[4];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) mx4[k4] = fmax3(sr[k4], sr[4 + k4], sr[8 + k4]);
+#pragma unroll
+                for (int e = 12; e + 8 <= C::NCHK * 32; e += 8)
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) mx4[k4] = fmax3(mx4[k4], sr[e + k4], sr[e + 4 + k4]);
+#pragma unroll
+                for (int e = 12 + ((C::NCHK * 32 - 12) / 8) * 8; e < C::NCHK * 32; e += 4)
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) mx4[k4] = fmaxf(mx4[k4], sr[e + k4]);
+                const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
                 const float m = mx * a.scale_log2;
                 const float ref = (mx == -CUDART_INF_F) ? 0.f : m;
                 const float2 nr2 = make_float2(-ref, -ref);
                 float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
+                // P = 2^(s*scale*log2e - m) as bf16 pairs over the first
+                // KEYS/2 columns of S (O is divided by the row sum in the
+                // epilogue); columns of chunks this warp cannot see are zero
+                uint32_t pk[C::NCHK * 16];
 #pragma unroll
                 for (int e = 0; e < C::NCHK * 32; e += 2) {
                     float2 y = fma2(make_float2(sr[e], sr[e + 1]), sc2, nr2);
-                    if ((e / 2) % NB_POLY_EVERY == NB_POLY_EVERY - 1) {
-                        y = exp2_poly2(y);
-                    } else {
-                        y.x = ex2_approx(y.x);
-                        y.y = ex2_approx(y.y);
-                    }
+                    y.x = ex2_approx(y.x);
+                    y.y = ex2_approx(y.y);
                     if (e & 2) acc2b = add2(acc2b, y);
                     else acc2 = add2(acc2, y);
-                    sr[e] = y.x;
-                    sr[e + 1] = y.y;
+                    pk[e / 2] = pack_bf16x2(y.x, y.y);
                 }
                 const float2 tot = add2(acc2, acc2b);
                 const float l = tot.x + tot.y;
                 const float inv = (l > 0.f) ? 1.f / l : 0.f;
-                // P = e / l as bf16 pairs over the first KEYS/2 columns of S;
-                // columns of chunks this warp cannot see are zero
                 uint32_t zero[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) zero[e] = 0u;
@@ -337,20 +377,14 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
                     tmem_st16u(s_base + cu * 16, zero);
                 }
 #pragma unroll
-                for (int cc = 0; cc < C::NCHK; ++cc) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(sr[cc * 32 + 2 * e] * inv, sr[cc * 32 + 2 * e + 1] * inv);
-                    tmem_st16u(s_base + (quarter + cc) * 16, pk);
-                }
+                for (int cc = 0; cc < C::NCHK; ++cc) tmem_st16u(s_base + (quarter + cc) * 16, pk + cc * 16);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->p_full[x]);
 
                 // ---- epilogue: O is final once this job's PV completes ----
-                const int h = un.hk * G + g;
+                const int h = un.h0 + g;
                 if (a.lse && row_real)
                     a.lse[((long long)un.b * a.Hq + h) * a.T + i] =
                         (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -364,14 +398,14 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
                     tmem_ld16(o_base + cc * 16, ov);
                     tmem_ld_wait_dep16(ov);
                     uint4 pk0, pk1;
-                    pk0.x = pack_bf16x2(ov[0], ov[1]);
-                    pk0.y = pack_bf16x2(ov[2], ov[3]);
-                    pk0.z = pack_bf16x2(ov[4], ov[5]);
-                    pk0.w = pack_bf16x2(ov[6], ov[7]);
-                    pk1.x = pack_bf16x2(ov[8], ov[9]);
-                    pk1.y = pack_bf16x2(ov[10], ov[11]);
-                    pk1.z = pack_bf16x2(ov[12], ov[13]);
-                    pk1.w = pack_bf16x2(ov[14], ov[15]);
+                    pk0.x = pack_bf16x2(ov[0] * inv, ov[1] * inv);
+                    pk0.y = pack_bf16x2(ov[2] * inv, ov[3] * inv);
+                    pk0.z = pack_bf16x2(ov[4] * inv, ov[5] * inv);
+                    pk0.w = pack_bf16x2(ov[6] * inv, ov[7] * inv);
+                    pk1.x = pack_bf16x2(ov[8] * inv, ov[9] * inv);
+                    pk1.y = pack_bf16x2(ov[10] * inv, ov[11] * inv);
+                    pk1.z = pack_bf16x2(ov[12] * inv, ov[13] * inv);
+                    pk1.w = pack_bf16x2(ov[14] * inv, ov[15] * inv);
                     if (row_real) {
                         reinterpret_cast<uint4 *>(dst + cc * 16)[0] = pk0;
                         reinterpret_cast<uint4 *>(dst + cc * 16)[1] = pk1;
@@ -392,13 +426,15 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
     }
 }
 
-template <int D, int PAD>
+template <int D, int PAD, int HP>
 cudaError_t launch_narrow_dp(const TcPrefillArgs &a, cudaStream_t s)
 {
-    using C = NCfg<D, PAD>;
+    using C = NCfg<D, PAD, HP>;
+    // HP adjacent heads as one row of HP*D elements
     CUtensorMap mq, mk, mv;
-    if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq, D, NB_BM) || !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv, D, C::KEYS) ||
-        !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv, D, C::KEYS))
+    if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq / HP, C::RD, NB_BM) ||
+        !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv / HP, C::RD, C::KEYS) ||
+        !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv / HP, C::RD, C::KEYS))
         return cudaErrorInvalidValue;
     static bool attr_set[64] = {};
     static int n_sm[64] = {};
@@ -406,17 +442,25 @@ cudaError_t launch_narrow_dp(const TcPrefillArgs &a, cudaStream_t s)
     cudaGetDevice(&dev);
     if (dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(swa_prefill_narrow_kernel<D, PAD>,
+        cudaError_t e = cudaFuncSetAttribute(swa_prefill_narrow_kernel<D, PAD, HP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if ((e = cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    const long long units = (long long)a.B * a.Hkv * ((a.T + NB_BM - 1) / NB_BM);
+    // a unit takes all G query heads of its tile (one K/V load) unless that
+    // leaves fewer than ~6 units per SM: then the heads are split in halves
+    // (quarters, ...), trading an L2 re-read of K/V for a shorter tail
+    const int G = HP * (a.Hq / a.Hkv);
+    long long units = (long long)a.B * (a.Hkv / HP) * ((a.T + NB_BM - 1) / NB_BM);
+    int n_slice = 1;
+    if (HP == 1)
+        while (G % (2 * n_slice) == 0 && units * n_slice < 6LL * n_sm[dev]) n_slice *= 2;
+    units *= n_slice;
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int grid = (int)(units < n_sm[dev] ? units : n_sm[dev]);
-    swa_prefill_narrow_kernel<D, PAD><<<grid, NB_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, a, (int)units);
+    swa_prefill_narrow_kernel<D, PAD, HP><<<grid, NB_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, a, (int)units, n_slice);
     return cudaGetLastError();
 }
 
@@ -430,8 +474,16 @@ bool prefill_narrow_applies(int d, const TcPrefillArgs &a)
 cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s)
 {
     if (!prefill_narrow_applies(d, a)) return cudaErrorInvalidValue;
-    if (d == 32) return a.left <= 31 ? launch_narrow_dp<32, 32>(a, s) : launch_narrow_dp<32, 64>(a, s);
-    return a.left <= 31 ? launch_narrow_dp<64, 32>(a, s) : launch_narrow_dp<64, 64>(a, s);
+    if (d == 32) {
+        // one query head per kv head and an even head count: two adjacent
+        // heads per tile row, so a unit has two jobs and its loads half the
+        // rows (with larger groups a unit already has several jobs, and
+        // single-head rows with sliced units measured faster)
+        if (a.Hkv % 2 == 0 && a.Hq == a.Hkv)
+            return a.left <= 31 ? launch_narrow_dp<32, 32, 2>(a, s) : launch_narrow_dp<32, 64, 2>(a, s);
+        return a.left <= 31 ? launch_narrow_dp<32, 32, 1>(a, s) : launch_narrow_dp<32, 64, 1>(a, s);
+    }
+    return a.left <= 31 ? launch_narrow_dp<64, 32, 1>(a, s) : launch_narrow_dp<64, 64, 1>(a, s);
 }
 
 }  // namespace swa

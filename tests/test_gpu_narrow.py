@@ -32,27 +32,38 @@ def test_narrow_windows(d, W, T):
     assert max_err(lse, ref_lse) <= 2e-2
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (3, 1), (6, 2), (8, 1), (5, 5)])
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (3, 1), (6, 2), (8, 1), (5, 5), (4, 4), (6, 6)])
 @pytest.mark.parametrize("W", [20, 60])
-def test_narrow_group_sizes(Hq, Hkv, W):
-    o, lse, ref_o, ref_lse = run(1, 300, Hq, Hkv, 64, W, seed=Hq * 10 + Hkv + W)
-    assert max_err(o, ref_o) <= 2e-2
-    assert max_err(lse, ref_lse) <= 2e-2
-
-
-@pytest.mark.parametrize("d,W", [(32, 32), (64, 64)])
-def test_narrow_more_units_than_sms(d, W):
-    # 3 * 8 * 16 = 384 units of (batch, kv head, tile): every CTA loops
-    o, lse, ref_o, ref_lse = run(3, 2000, 16, 8, d, W, seed=d + W)
-    assert max_err(o, ref_o) <= 2e-2
-    assert max_err(lse, ref_lse) <= 2e-2
-
-
 @pytest.mark.parametrize("d", [32, 64])
-def test_narrow_window_one_returns_v_exactly(d):
-    q, k, v = wl.prefill_inputs(1, 300, 4, 2, d, torch.bfloat16, 8)
+def test_narrow_group_sizes(Hq, Hkv, W, d):
+    # d = 32 with one query head per kv head and an even head count loads
+    # two heads per tile row
+    o, lse, ref_o, ref_lse = run(1, 300, Hq, Hkv, d, W, seed=Hq * 10 + Hkv + W + d)
+    assert max_err(o, ref_o) <= 2e-2
+    assert max_err(lse, ref_lse) <= 2e-2
+
+
+@pytest.mark.parametrize("W", [1, 32, 33, 64])
+@pytest.mark.parametrize("T", [129, 390])
+def test_narrow_paired_heads(W, T):
+    o, lse, ref_o, ref_lse = run(2, T, 8, 8, 32, W, seed=W * 7 + T)
+    assert max_err(o, ref_o) <= 2e-2
+    assert max_err(lse, ref_lse) <= 2e-2
+
+
+@pytest.mark.parametrize("d,W,Hq,Hkv", [(32, 32, 16, 8), (64, 64, 16, 8), (32, 50, 16, 16)])
+def test_narrow_more_units_than_sms(d, W, Hq, Hkv):
+    # 3 * 8 * 16 = 384 units of (batch, kv heads, tile) or more: every CTA loops
+    o, lse, ref_o, ref_lse = run(3, 2000, Hq, Hkv, d, W, seed=d + W + Hq)
+    assert max_err(o, ref_o) <= 2e-2
+    assert max_err(lse, ref_lse) <= 2e-2
+
+
+@pytest.mark.parametrize("d,Hq,Hkv", [(32, 4, 2), (64, 4, 2), (32, 4, 4)])
+def test_narrow_window_one_returns_v_exactly(d, Hq, Hkv):
+    q, k, v = wl.prefill_inputs(1, 300, Hq, Hkv, d, torch.bfloat16, 8)
     o = swa.swa_prefill(q.to(dev()), k.to(dev()), v.to(dev()), 1)
-    assert torch.equal(o.cpu(), v.repeat_interleave(2, dim=2))
+    assert torch.equal(o.cpu(), v.repeat_interleave(Hq // Hkv, dim=2))
 
 
 def test_narrow_output_untouched_outside_rows():
