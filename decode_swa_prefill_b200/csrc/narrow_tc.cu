@@ -13,8 +13,7 @@
 // Persistent CTAs, one per SM (two TMEM buffers take all 512 columns), walk
 // units of (batch, kv head, query tile[, slice of the query heads]) with a
 // stride of the grid size; the query heads of a unit share its K/V tile and
-// are its jobs.  Job j uses
-// TMEM buffer j & 1:
+// are its jobs.  Job j uses TMEM buffer j & 1:
 //   O[b]  columns 256b .. 256b+d-1       fp32 output of the job
 //   S[b]  columns 256b+64 .. +128+PAD-1  fp32 scores; P (bf16 pairs) over
 //                                        its first (128+PAD)/2 columns
@@ -22,15 +21,16 @@
 //   warps 0-3  softmax + epilogue of the even jobs (thread r = row r = TMEM
 //              lane r), warps 4-7 the same for the odd jobs
 //   warp 8     producer: TMA loads of K, V (128+PAD rows) per unit and of Q
-//              (128 rows) per job into rings of 2 and 4 stages
+//              (128 rows) per job (per pair of jobs with paired head rows)
+//              into rings of 3-4 and 4-8 stages
 //   warp 9     TMEM allocator and MMA issuer (lane 0): QK^T of job j, then
 //              PV of job j-1, so a QK^T runs while the previous job's
 //              softmax works.  S[b] is rewritten once the PV that read P[b]
 //              has completed, O[b] once the epilogue two jobs back has read
 //              it: the epilogue is off the MMA's critical path.
 // A warp only computes the 32-key chunks its rows can see (two for PAD 32,
-// three for PAD 64) and writes zeros to the rest of its P columns.  The
-// softmax is issue-bound, so every exponential runs on the MUFU.
+// three for PAD 64) and writes zeros to the rest of its P columns; every
+// exponential runs on the MUFU.
 //
 // Every mbarrier wait is bounded: on expiry the CTA records
 // SWA_STATUS_TIMEOUT, drains its in-flight copies and MMAs with a second
@@ -85,6 +85,7 @@ struct NCfg {
     static_assert(QTILE % 1024 == 0 && KVTILE % 1024 == 0, "1 KiB aligned stages");
     static_assert(SMEM_BYTES <= 227 * 1024, "fits one SM");
     static_assert(2 * (SMEM_BYTES + 1024) > 228 * 1024, "never two CTAs per SM");
+    static_assert(QST <= NB_QST_MAX && KVST <= NB_KVST_MAX, "barrier arrays");
 };
 
 __host__ __device__ constexpr uint32_t nb_col_o(int b) { return 256u * b; }
