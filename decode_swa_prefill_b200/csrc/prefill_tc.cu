@@ -210,16 +210,19 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs
     } else {
         bid -= n_mode1;
         w.mode = 0;
+        // query tiles in descending order: the CTAs the hardware starts last
+        // are the short ones at the start of a causal sequence, which fill
+        // the tail of the grid instead of full-window CTAs
         if (pair_heads) {
             const int hp = bid % (a.Hq / 2);
-            const int qt = (bid / (a.Hq / 2)) % nqt;
+            const int qt = nqt - 1 - (bid / (a.Hq / 2)) % nqt;
             w.b = bid / ((a.Hq / 2) * nqt);
             for (int x = 0; x < 2; ++x)
                 w.q[x] = QTile{2 * hp + x, qt * BM, 0, min(BM, a.T - qt * BM), 0, 0, true};
         } else {
             const int h = bid % a.Hq;
             const int nqp = (nqt + 1) / 2;
-            const int qp = (bid / a.Hq) % nqp;
+            const int qp = nqp - 1 - (bid / a.Hq) % nqp;
             w.b = bid / (a.Hq * nqp);
             for (int x = 0; x < 2; ++x) {
                 const int qt = 2 * qp + x;
