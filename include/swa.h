@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
     SWA_OK = 0,
     SWA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0 ... */
-    SWA_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for (e.g. d) */
+    SWA_ERR_UNSUPPORTED = 2, /* valid request the library has no kernel for (e.g. d) */
     SWA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     SWA_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired; its outputs are invalid */
 } swa_status;
