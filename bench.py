@@ -177,6 +177,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------ distributed --
 
+def relaunch_command(gpus, argv, port):
+    """The torchrun command line that runs this script as `gpus` ranks (one
+    process per GPU) with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(gpus),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -292,7 +308,8 @@ def gpu_arm(args, world, rank, local):
 
     # ---- end to end through the public API with host buffers ----
     e2e = e2e_arm(st, args, world, dev, step_flops)
-    extra = tinymistral_arm(swa, dev, args)
+    extra, tiny_o = tinymistral_arm(swa, dev, args)
+    toy, toy_o = toy_arm(swa, dev, args)
     chunk = chunk_arm(swa, dev, args)
     sinks = sinks_arm(swa, dev, args, load_peaks()[0])
     dilated = dilated_arm(swa, dev, args, load_peaks()[0])
@@ -325,6 +342,7 @@ def gpu_arm(args, world, rank, local):
                            "flops": acc["f_lf"]},
             "append": {"us": round(avg["append"] * 1e3, 2)},
             "tinymistral_prefill": extra,
+            "toy_f32": toy,
             "chunk_prefill": chunk,
             "sinks": sinks,
             "dilated": dilated,
@@ -346,24 +364,32 @@ def gpu_arm(args, world, rank, local):
         "gpu_launches": st.launches_per_step * args.steps,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args, world)
+        # the GPU outputs of the five configurations, for the parity check
+        # the CPU-baseline leg runs next to its timing
+        outs = {"prefill": st.o.cpu(), "longformer": st.lo.cpu(), "decode": st.do.cpu(),
+                "tinymistral": tiny_o.cpu(), "toy": toy_o.cpu()}
+        line["cpu_baseline"], line["max_abs_err"] = cpu_baseline(args, world, st.host, outs)
     return line
 
 
 def tinymistral_arm(swa, dev, args):
     """TinyMistral-shaped prefill (B=4, T=2048, 32/8 heads, d=32, W=32): HBM
     bound (25 FLOP per byte), not part of the step.  Its 42 MB fit in L2, so
-    L2 is flushed (256 MB write) before every timed launch."""
+    L2 is flushed before every timed launch by READING a 256 MB buffer: a
+    written flush buffer would leave ~126 MB of dirty lines whose write-back
+    then competes with the timed launch."""
     w = wl.TINYMISTRAL
     inp = {k: v.to(dev) for k, v in wl.make(w).items()}
     o = torch.empty_like(inp["q"])
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(32 << 20, dtype=torch.float64, device=dev)   # 256 MB, written once
+    sink = torch.empty((), dtype=torch.float64, device=dev)
+    torch.cuda.synchronize()
     peaks, _ = load_peaks()
     flops = causal_pairs(w.T, w.W) * w.B * w.Hq * 4 * w.d
     nbytes = w.B * w.T * (2 * w.Hq + 2 * w.Hkv) * w.d * 2
     times = []
     for i in range(args.warmup + max(10, args.steps // 2)):
-        flush.zero_()
+        torch.sum(flush, out=sink)       # read sweep: evicts L2, leaves clean lines
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W, o=o)
@@ -375,8 +401,27 @@ def tinymistral_arm(swa, dev, args):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
             "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "bytes": nbytes, "flops": flops,
-            "l2": "flushed before each launch", "kernel": "swa_prefill_narrow_kernel",
-            "traffic": recorded_traffic("tinymistral")}
+            "l2": "flushed before each launch by a 256 MB read sweep", "kernel": "swa_prefill_narrow_kernel",
+            "traffic": recorded_traffic("tinymistral")}, o
+
+
+def toy_arm(swa, dev, args):
+    """The fp32 toy configuration (B=1, T=16, W=4, d=64): launch-latency
+    bound, reported in microseconds only."""
+    w = wl.TOY
+    inp = {k: v.to(dev) for k, v in wl.make(w).items()}
+    o = torch.empty_like(inp["q"])
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W, o=o)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    return {"us": round(sum(times) / len(times) * 1e3, 2), "workload": w.name, "dtype": "f32",
+            "kernel": "prefill_f32_kernel"}, o
 
 
 def chunk_pairs(n, W, p0):
@@ -591,7 +636,15 @@ def e2e_arm(st, args, world, dev, step_flops):
 
 # ------------------------------------------------------- oracle (CPU) --
 
-def oracle_sample(budget_s, seed=0):
+def f64_inputs():
+    """The step's inputs as fp64 numpy arrays (the oracle's own input type),
+    converted once so that the timed oracle calls do not convert them."""
+    P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
+    f = lambda d: {k: (v.double().numpy() if v.is_floating_point() else v.numpy()) for k, v in d.items()}
+    return f(wl.make(P)), f(wl.make(L)), f(wl.make(D))
+
+
+def oracle_sample(budget_s, seed=0, inputs=None):
     """Run the fp64 oracle on a seeded row sample of every component of the
     step; returns (in-window FLOPs computed, seconds, threads)."""
     import oracle
@@ -599,9 +652,7 @@ def oracle_sample(budget_s, seed=0):
     P, L, D = wl.MISTRAL_PREFILL, wl.LONGFORMER, wl.MISTRAL_DECODE
     threads = oracle.default_threads()
     flops, secs = 0, 0.0
-    hp = wl.make(P)
-    hl = wl.make(L)
-    hd = wl.make(D)
+    hp, hl, hd = inputs if inputs is not None else f64_inputs()
     # rows per component in proportion to their share of a step's FLOPs
     plan = [("prefill", 0.80), ("longformer", 0.15), ("decode", 0.05)]
     for name, share in plan:
@@ -621,7 +672,7 @@ def oracle_sample(budget_s, seed=0):
                 i = rng.integers(0, L.T, 64)
                 oracle.swa_prefill_global(hl["q"], hl["k"], hl["v"], hl["global_idx"], L.W,
                                           rows=oracle.row_ids(b, h, i, L.Hq, L.T))
-                gi = hl["global_idx"].numpy()
+                gi = hl["global_idx"]
                 for bb, ii in zip(b, i):
                     row = gi[bb]
                     if ii in row:
@@ -640,13 +691,63 @@ def oracle_sample(budget_s, seed=0):
     return flops, secs, threads
 
 
-def cpu_baseline(args, world):
-    flops, secs, threads = oracle_sample(args.cpu_seconds)
-    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+def parity_errors(host, outs, seed=7):
+    """Max abs error of the bench's own GPU outputs against the fp64 oracle:
+    every row of the TinyMistral, toy and decode configurations, and for the
+    Mistral and Longformer prefills a seeded sample of rows of every head
+    (the last row of each head, 64 random rows, and every global row)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    hp, hl, hd = host
+    P, L = wl.MISTRAL_PREFILL, wl.LONGFORMER
+    err = {}
+
+    def mx(got, ref):
+        return float(np.abs(np.asarray(got, dtype=np.float64) - ref).max())
+
+    b, h, i = [], [], []
+    for hh in range(P.Hq):
+        rows = np.concatenate([[P.T - 1], rng.integers(0, P.T, 64)])
+        b += [0] * len(rows); h += [hh] * len(rows); i += rows.tolist()
+    b, h, i = map(np.array, (b, h, i))
+    ref, _ = oracle.swa_prefill(hp["q"], hp["k"], hp["v"], P.W, rows=oracle.row_ids(b, h, i, P.Hq, P.T))
+    err["mistral7b_prefill"] = mx(outs["prefill"][b, i, h].float().numpy(), ref)
+    b, h, i = [], [], []
+    for bb in range(L.B):
+        for hh in range(L.Hq):
+            rows = np.concatenate([[L.T - 1], rng.integers(0, L.T, 64), hl["global_idx"][bb]])
+            b += [bb] * len(rows); h += [hh] * len(rows); i += rows.tolist()
+    b, h, i = map(np.array, (b, h, i))
+    ref, _ = oracle.swa_prefill_global(hl["q"], hl["k"], hl["v"], hl["global_idx"], L.W,
+                                       rows=oracle.row_ids(b, h, i, L.Hq, L.T))
+    err["longformer_prefill"] = mx(outs["longformer"][b, i, h].float().numpy(), ref)
+    # decode: the bench appended the new token at pos before every decode
+    kc, vc, _ = oracle.ring_append(hd["k_cache"], hd["v_cache"], hd["k_new"], hd["v_new"], hd["pos"])
+    ref, _ = oracle.swa_decode(hd["q"], kc, vc, hd["pos"])
+    err["mistral7b_decode"] = mx(outs["decode"].float().numpy(), ref)
+    for name, w in (("tinymistral", wl.TINYMISTRAL), ("toy", wl.TOY)):
+        t = wl.make(w)
+        ref, _ = oracle.swa_prefill(t["q"], t["k"], t["v"], w.W)
+        err[w.name] = mx(outs[name].float().numpy(), ref)
+    err["tolerance"] = {"bf16": 2e-2, "f32": 1e-5}
+    return err
+
+
+def cpu_baseline(args, world, host=None, outs=None):
+    """The fp64 oracle timed on the host cores on a bounded sample of the
+    step; with the bench's GPU outputs it also reports their max abs error
+    against the oracle per configuration (not timed)."""
+    inputs = f64_inputs()
+    flops, secs, threads = oracle_sample(args.cpu_seconds, inputs=inputs)
+    base = {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
             "kind": "oracle",
             "sample": "fp64 oracle on seeded row samples of the same step (about %.0f s: "
                       "Mistral prefill rows past W, Longformer rows, decode sequences), scaled by "
-                      "their in-window FLOPs" % args.cpu_seconds}
+                      "their in-window FLOPs; inputs converted to fp64 once, before the timing"
+                      % args.cpu_seconds}
+    if outs is None:
+        return base
+    return base, parity_errors(inputs, outs)
 
 
 def reference_arm(args, world, rank):
@@ -656,10 +757,11 @@ def reference_arm(args, world, rank):
         return None
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
     flops_total, secs_total, threads = 0, 0.0, 1
+    inputs = f64_inputs()
     for s in range(args.warmup):
-        oracle_sample(min(per_step, 1.0), seed=1000 + s)
+        oracle_sample(min(per_step, 1.0), seed=1000 + s, inputs=inputs)
     for s in range(args.steps):
-        f, t, threads = oracle_sample(per_step, seed=s)
+        f, t, threads = oracle_sample(per_step, seed=s, inputs=inputs)
         flops_total += f
         secs_total += t
     v = flops_total / secs_total / 1e12
@@ -731,6 +833,14 @@ def main():
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # not under torchrun yet: become `gpus` ranks, one process per GPU
+        sys.stdout.flush()
+        os.execv(sys.executable, relaunch_command(args.gpus, sys.argv[1:], free_port()))
+    if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE is %s" % (args.gpus, os.environ.get("WORLD_SIZE", "1")))
     if args.impl == "reference":
         # rank 0 alone runs the oracle; other ranks exit without work
         world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -140,18 +140,16 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
     return o
 
 
-def swa_prefill_varlen(q, k, v, cu_seqlens, W, max_seqlen=None, scale=None, o=None, lse=None, stream=None):
+def swa_prefill_varlen(q, k, v, cu_seqlens, W, max_seqlen, scale=None, o=None, lse=None, stream=None):
     """Causal window over packed sequences q [total,Hq,d], k/v [total,Hkv,d];
-    cu_seqlens int32 [nseq+1] on the device.  max_seqlen (the longest
-    sequence) is read from cu_seqlens when not given."""
+    cu_seqlens int32 [nseq+1] on the device; max_seqlen is the longest
+    sequence (a host integer the caller knows, like the offsets themselves)."""
     _dev_contig(q, k, v, o, lse, cu_seqlens)
     total, Hq, d = q.shape
     Hkv = k.shape[1]
     _need(k.shape == (total, Hkv, d) and v.shape == k.shape, "k/v shape")
     _need(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1, "cu_seqlens int32 [nseq+1]")
     nseq = cu_seqlens.numel() - 1
-    if max_seqlen is None:
-        max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item()) if nseq > 0 else 0
     if o is None:
         o = torch.empty_like(q)
     scale = d ** -0.5 if scale is None else scale

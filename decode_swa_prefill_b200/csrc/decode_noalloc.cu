@@ -54,6 +54,7 @@ extern "C" swa_status swa_decode_noalloc(const void *q, const void *k_cache, con
                                          const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
                                          swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_decode_noalloc");
     if (dt != SWA_DTYPE_BF16 && dt != SWA_DTYPE_F32) return SWA_ERR_INVALID_ARG;
     if (B < 0 || Hq < 1 || Hkv < 1 || W < 1 || d < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;

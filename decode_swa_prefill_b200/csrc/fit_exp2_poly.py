@@ -8,8 +8,8 @@ small factor of the minimax polynomial).  The kernel applies 2^j by adding j
 to the exponent field of p(f).
 
 Run to print the coefficients (highest degree first) and the worst relative
-error over a dense grid; the coefficients in prefill_tc.cu were produced by
-`python fit_exp2_poly.py 3`.
+error over a dense grid; the coefficients of exp2_poly2 in ptx.cuh were
+produced by `python fit_exp2_poly.py 3`.
 """
 import sys
 

@@ -437,18 +437,15 @@ cudaError_t launch_narrow_dp(const TcPrefillArgs &a, cudaStream_t s)
         !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv / HP, C::RD, C::KEYS) ||
         !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv / HP, C::RD, C::KEYS))
         return cudaErrorInvalidValue;
-    static bool attr_set[64] = {};
-    static int n_sm[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(swa_prefill_narrow_kernel<D, PAD, HP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        if ((e = cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    static DeviceOnce once;
+    int n_sm = 0;
+    cudaError_t e = once.get(
+        [&](int) {
+            return cudaFuncSetAttribute(swa_prefill_narrow_kernel<D, PAD, HP>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        },
+        &n_sm);
+    if (e != cudaSuccess) return e;
     // a unit takes all G query heads of its tile (one K/V load) unless that
     // leaves fewer than ~6 units per SM: then the heads are split in halves
     // (quarters, ...), trading an L2 re-read of K/V for a shorter tail
@@ -456,11 +453,11 @@ cudaError_t launch_narrow_dp(const TcPrefillArgs &a, cudaStream_t s)
     long long units = (long long)a.B * (a.Hkv / HP) * ((a.T + NB_BM - 1) / NB_BM);
     int n_slice = 1;
     if (HP == 1)
-        while (G % (2 * n_slice) == 0 && units * n_slice < 6LL * n_sm[dev]) n_slice *= 2;
+        while (G % (2 * n_slice) == 0 && units * n_slice < 6LL * n_sm) n_slice *= 2;
     units *= n_slice;
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const int grid = (int)(units < n_sm[dev] ? units : n_sm[dev]);
+    const int grid = (int)(units < n_sm ? units : n_sm);
     swa_prefill_narrow_kernel<D, PAD, HP><<<grid, NB_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, a, (int)units, n_slice);
     return cudaGetLastError();
 }

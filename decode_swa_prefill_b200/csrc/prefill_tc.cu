@@ -1005,19 +1005,18 @@ cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cu
     // sinks: no global positions but g > 0 (causal window plus the first g
     // positions)
     const bool sinks = !RING && a.gidx == nullptr && a.g > 0;
-    static bool attr_set[64][2] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev][sinks]) {
-        cudaError_t e = RING    ? cudaFuncSetAttribute(swa_prefill_ring_kernel<D>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
-                        : sinks ? cudaFuncSetAttribute(swa_prefill_sinks_kernel<D>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
-                                : cudaFuncSetAttribute(swa_prefill_tc_kernel<D>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set[dev][sinks] = true;
-    }
+    static DeviceOnce once[2];
+    cudaError_t e = once[sinks].get(
+        [&](int) {
+            return RING    ? cudaFuncSetAttribute(swa_prefill_ring_kernel<D>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                   : sinks ? cudaFuncSetAttribute(swa_prefill_sinks_kernel<D>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES)
+                           : cudaFuncSetAttribute(swa_prefill_tc_kernel<D>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        },
+        nullptr);
+    if (e != cudaSuccess) return e;
     const int G = a.Hq / a.Hkv;
     const bool pair_heads = (G % 2) == 0;
     const int nqt = (a.T + BM - 1) / BM;
@@ -1054,15 +1053,14 @@ cudaError_t launch_varlen_d(const TcPrefillArgs &a, const VarlenArgs &vl, cudaSt
     if (!make_map<D>(&mq, a.q, 1, a.T, a.Hq, BM) || !make_map<D>(&mk, a.k, 1, a.T, a.Hkv, BN) ||
         !make_map<D>(&mv, a.v, 1, a.T, a.Hkv, BN) || !make_map<D>(&mo, a.o, 1, a.T, a.Hq, BM))
         return cudaErrorInvalidValue;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(swa_prefill_varlen_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    static DeviceOnce once;
+    cudaError_t e = once.get(
+        [&](int) {
+            return cudaFuncSetAttribute(swa_prefill_varlen_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::SMEM_BYTES);
+        },
+        nullptr);
+    if (e != cudaSuccess) return e;
     const int G = a.Hq / a.Hkv;
     const bool pair_heads = (G % 2) == 0;
     const int nqt = (vl.max_len + BM - 1) / BM;

@@ -372,12 +372,15 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b)
 // Cody-Waite range reduction 2^x = 2^j * 2^f, j = round(x), f in [-1/2, 1/2]
 // (rounding by adding 1.5*2^23), a cubic for 2^f from a weighted least-squares
 // fit on Chebyshev nodes (fit_exp2_poly.py; max relative error 7.7e-5, far
-// below bf16 resolution), and j added to the exponent field.  x is clamped to
-// -125 so the result stays a normal float (2^-125 stands in for 0).
-__device__ __forceinline__ float2 exp2_poly2(float2 x)
+// below bf16 resolution), and j added to the exponent field.  Arguments below
+// -125 (a masked score is -inf) give exactly 0, as ex2.approx does for -inf:
+// the reduction runs on the argument clamped to -125 so the exponent field
+// never underflows, and a select replaces those results by 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x0)
 {
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
+    float2 x;
+    x.x = fmaxf(x0.x, -125.f);
+    x.y = fmaxf(x0.y, -125.f);
     const float2 t = add2(x, make_float2(12582912.f, 12582912.f));
     const float2 j = add2(t, make_float2(-12582912.f, -12582912.f));
     const float2 f = fma2(j, make_float2(-1.f, -1.f), x);
@@ -386,8 +389,8 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x)
     p = fma2(p, f, make_float2(6.932762265e-01f, 6.932762265e-01f));
     p = fma2(p, f, make_float2(9.999289513e-01f, 9.999289513e-01f));
     float2 r;
-    r.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
-    r.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+    r.x = x0.x < -125.f ? 0.f : __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+    r.y = x0.y < -125.f ? 0.f : __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
     return r;
 }
 

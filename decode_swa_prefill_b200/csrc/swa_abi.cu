@@ -130,6 +130,7 @@ void swa_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns = ns > 0 ? n
 swa_status swa_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int T, int Hq,
                        int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill");
     swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK || B == 0 || T == 0) return st;
     const int left = W - 1 < T ? W - 1 : T;  // a window wider than T is T
@@ -154,6 +155,7 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
                               const int32_t *global_idx, int g, int B, int T, int Hq, int Hkv, int d, int W,
                               float scale, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill_global");
     swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK) return st;
     if (g < 0 || g > T) return SWA_ERR_INVALID_ARG;
@@ -187,6 +189,7 @@ swa_status swa_prefill_dilated(const void *q, const void *k, const void *v, void
                                int symmetric, int B, int T, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
                                void *workspace, size_t workspace_bytes, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill_dilated");
     swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK) return st;
     if (dil < 1 || (symmetric != 0 && symmetric != 1)) return SWA_ERR_INVALID_ARG;
@@ -243,6 +246,7 @@ swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void 
                               const int32_t *cu_seqlens, int nseq, int total, int max_seqlen, int Hq, int Hkv, int d,
                               int W, float scale, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill_varlen");
     swa_status st = check_prefill(q, k, v, o, lse, 1, total, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK) return st;
     if (nseq < 0 || max_seqlen < 0 || max_seqlen > total) return SWA_ERR_INVALID_ARG;
@@ -271,6 +275,7 @@ swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void 
 swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink, int B,
                              int T, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill_sinks");
     swa_status st = check_prefill(q, k, v, o, lse, B, T, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK) return st;
     if (n_sink < 0) return SWA_ERR_INVALID_ARG;
@@ -299,6 +304,7 @@ swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *
                              const void *v_cache, const int32_t *pos, int B, int n, int Hq, int Hkv, int d, int W,
                              float scale, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_prefill_chunk");
     swa_status st = check_prefill(q, k, v, o, lse, B, n, Hq, Hkv, d, W, scale, dt);
     if (st != SWA_OK || B == 0 || n == 0) return st;
     if (!k_cache || !v_cache || !pos) return SWA_ERR_INVALID_ARG;
@@ -328,6 +334,7 @@ swa_status swa_prefill_chunk(const void *q, const void *k, const void *v, void *
 swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, const void *v_new, const int32_t *pos,
                             int32_t *slot_out, int B, int n, int Hkv, int d, int W, swa_dtype dt, void *stream)
 {
+    SWA_NVTX_RANGE("swa_cache_append");
     if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
     if (B < 0 || n < 0 || Hkv < 1 || d < 1 || W < 1) return SWA_ERR_INVALID_ARG;
     if ((d * elt_size(dt)) % 16 != 0) return SWA_ERR_UNSUPPORTED;
@@ -395,6 +402,7 @@ swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, v
                       const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
                       void *workspace, size_t workspace_bytes, void *stream)
 {
+    SWA_NVTX_RANGE("swa_decode");
     return decode_impl(q, k_cache, v_cache, nullptr, nullptr, 0, o, lse, pos, B, Hq, Hkv, d, W, scale, dt, workspace,
                        workspace_bytes, stream);
 }
@@ -404,6 +412,7 @@ swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_ca
                             int Hkv, int d, int W, float scale, swa_dtype dt, void *workspace, size_t workspace_bytes,
                             void *stream)
 {
+    SWA_NVTX_RANGE("swa_decode_sinks");
     return decode_impl(q, k_cache, v_cache, k_sink, v_sink, n_sink, o, lse, pos, B, Hq, Hkv, d, W, scale, dt,
                        workspace, workspace_bytes, stream);
 }
@@ -411,6 +420,7 @@ swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_ca
 swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric, const int32_t *global_idx, int g,
                            void *stream)
 {
+    SWA_NVTX_RANGE("swa_mask_export");
     if (T < 0 || T > 65536 || W < 1 || (symmetric != 0 && symmetric != 1)) return SWA_ERR_INVALID_ARG;
     if (g < 0 || g > T || (g > 0 && !symmetric)) return SWA_ERR_INVALID_ARG;
     if (T == 0) return SWA_OK;

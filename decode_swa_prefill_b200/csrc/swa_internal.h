@@ -3,6 +3,21 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
+#include <nvtx3/nvToolsExt.h>
+
+// A named NVTX range around one C-ABI call, so a timeline (Nsight Systems,
+// ncu's NVTX filters) shows which call launched which kernels.  NVTX v3 is
+// header-only; without a tool attached each push/pop is a cheap no-op.
+struct SwaNvtxRange {
+    explicit SwaNvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~SwaNvtxRange() { nvtxRangePop(); }
+    SwaNvtxRange(const SwaNvtxRange &) = delete;
+    SwaNvtxRange &operator=(const SwaNvtxRange &) = delete;
+};
+#define SWA_NVTX_RANGE(name) SwaNvtxRange swa_nvtx_range_(name)
+
 // Device status word values (ordered: the worst one wins via atomicMax).
 #define SWA_STATUS_OK 0
 #define SWA_STATUS_BAD_INPUT 1
@@ -17,6 +32,38 @@ __host__ __device__ __forceinline__ bool band_contains(long long i, long long j,
 {
     return j >= i - left && j <= i + right;
 }
+
+// One-time setup per device of a kernel launcher (kernel attributes, the SM
+// count), safe when several host threads launch on the same device: the
+// first call for a device runs init(dev, &n_sm) under a mutex, later calls
+// read the stored SM count under the same mutex.
+class DeviceOnce {
+  public:
+    template <typename F>
+    cudaError_t get(F init, int *n_sm_out)
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMax) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (!done_[dev]) {
+            int n = 0;
+            if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+            if ((e = init(dev)) != cudaSuccess) return e;
+            n_sm_[dev] = n;
+            done_[dev] = true;
+        }
+        if (n_sm_out) *n_sm_out = n_sm_[dev];
+        return cudaSuccess;
+    }
+
+  private:
+    static constexpr int kMax = 64;
+    std::mutex mu_;
+    bool done_[kMax] = {};
+    int n_sm_[kMax] = {};
+};
 
 struct DeviceCtl {
     int *status;                 // device status word

@@ -18,7 +18,9 @@
  *
  * Conventions for every call:
  *  - Every buffer is owned by the caller and lives in device memory unless a
- *    parameter says otherwise.  The library never allocates device memory.
+ *    parameter says otherwise.  The library never allocates device memory
+ *    at run time; its device code holds two static arrays (a status word and
+ *    the 16 MiB scratch of swa_decode_noalloc) on each GPU it is loaded on.
  *  - Tensors are dense, row-major, 16-byte aligned, with the layouts given
  *    below (innermost dimension last).  B batch, T sequence length, Hq query
  *    heads, Hkv key/value heads (Hq % Hkv == 0; query head h reads kv head
@@ -230,14 +232,18 @@ swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_ca
  * its own, a plugin inside a runtime that owns all device memory, or a
  * serving loop where an allocation could block on the device.  The pages
  * have no counterpart of this call; it exists only for those callers.
- *   Arguments, layouts and results as swa_decode.
- *   Scratch: one static device array of 16 MiB, held by every GPU that loads
- *   this library until the process exits.  Sizes whose split partials
+ *   Arguments, layouts and results as swa_decode (bit for bit: the same
+ *   kernels with the same split count).
+ *   Scratch: one static device array of 16 MiB.  It is part of the library's
+ *   device code, so every process that loads this library holds it on every
+ *   GPU the library's kernels are loaded on, until the process exits, whether
+ *   or not it ever calls swa_decode_noalloc.  Sizes whose split partials
  *   (swa_decode_workspace_bytes) exceed 16 MiB are rejected with
  *   SWA_ERR_UNSUPPORTED before anything runs.  Nothing is allocated.
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current and keeps it for the
+ *   life of the process; make that first call before any stream capture, and
+ *   do not use this call on a device after cudaDeviceReset.
  *   All calls share the array: calls whose kernels overlap on the GPU (two
  *   streams, or two host threads on one device) race and give wrong results.
  *   Each call writes every scratch record it reads, so nothing is cleared

@@ -24,3 +24,14 @@ def max_err(got, ref):
 
 def tol_for(dtype):
     return BF16_TOL if dtype == torch.bfloat16 else F32_TOL
+
+
+def poison_unfilled(k_cache, v_cache, filled):
+    """Set to NaN every ring slot a sequence has not reached yet: slots
+    filled[b] .. W-1 of row b (CPU tensors, in place).  A reader that touches
+    one of them, even to mask it afterwards, turns its output into NaN."""
+    W = k_cache.shape[2]
+    for b, n in enumerate(int(x) for x in filled):
+        if n < W:
+            k_cache[b, :, n:] = float("nan")
+            v_cache[b, :, n:] = float("nan")

@@ -98,3 +98,44 @@ def test_reference_arm_only_rank0_works():
     out = mp.Manager().dict()
     mp.spawn(_ref_rank, args=(2, 0, out), nprocs=2, join=True)
     assert out[1] is None
+
+
+def _bench_env():
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["PYTHONPATH"] = bench.ROOT
+    return env
+
+
+def test_relaunch_command_is_one_rank_per_gpu():
+    cmd = bench.relaunch_command(4, ["--gpus", "4", "--steps", "2"], 12345)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert cmd[cmd.index("--nproc-per-node") + 1] == "4"
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "2"]
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    # --gpus 2 outside torchrun re-executes the script as two ranks; the
+    # reference arm (CPU only) then prints one line, from rank 0, that counts
+    # both ranks
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--impl",
+                          "reference", "--steps", "1", "--warmup", "3", "--cpu-seconds", "1"],
+                         capture_output=True, text=True, timeout=900, env=_bench_env())
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+    import sys
+    env = _bench_env()
+    env.update(WORLD_SIZE="3", RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2"],
+                         capture_output=True, text=True, timeout=300, env=env)
+    assert out.returncode != 0 and "WORLD_SIZE" in out.stderr

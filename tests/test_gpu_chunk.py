@@ -10,13 +10,16 @@ import torch
 import decode_swa_prefill_b200 as swa
 import oracle
 from decode_swa_prefill_b200 import workloads as wl
-from gpu_util import dev, max_err, tol_for
+from gpu_util import dev, max_err, poison_unfilled, tol_for
 
 pytestmark = pytest.mark.gpu
 
 
 def run_chunk(B, n, Hq, Hkv, d, W, pos, dtype, seed):
     q, k, v, kc, vc = wl.chunk_inputs(B, n, Hq, Hkv, d, W, dtype, seed)
+    # a ring holding positions 0..pos-1 has written only slots 0..pos-1 when
+    # pos < W: the others are NaN, and must never be read
+    poison_unfilled(kc, vc, [min(p, W) for p in pos])
     p = torch.tensor(pos, dtype=torch.int32)
     lse = torch.zeros(B, Hq, n, dtype=torch.float32, device=dev())
     o = swa.swa_prefill_chunk(q.to(dev()), k.to(dev()), v.to(dev()), kc.to(dev()), vc.to(dev()), p.to(dev()),
@@ -60,8 +63,8 @@ def test_sequence_chunk_by_chunk_equals_one_prefill(dtype, d):
     T = sum(sizes)
     q, k, v = wl.prefill_inputs(1, T, Hq, Hkv, d, dtype, seed=d)
     ref_o, _ = oracle.swa_prefill(q, k, v, W)
-    kc = torch.zeros(1, Hkv, W, d, dtype=dtype, device=dev())
-    vc = torch.zeros_like(kc)
+    kc = torch.full((1, Hkv, W, d), float("nan"), dtype=dtype, device=dev())   # never-written slots
+    vc = torch.full_like(kc, float("nan"))
     qd, kd, vd = q.to(dev()), k.to(dev()), v.to(dev())
     p = 0
     outs = []

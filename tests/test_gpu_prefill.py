@@ -67,6 +67,19 @@ def test_window_one_returns_v_exactly():
     assert torch.equal(o.cpu(), v.repeat_interleave(2, dim=2))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_masked_keys_weigh_exactly_zero(d):
+    # W = 1: in each key tile every key but one is masked for a row.  Odd
+    # keys carry 2^127, so a masked key given any weight at all (even the
+    # smallest normal float, 2^-126, times 2^127 is 2) would move an even
+    # row's output away from 1.0; the rows must return their own V exactly.
+    q, k, v = wl.prefill_inputs(1, 256, 2, 1, d, torch.bfloat16, 8)
+    v = torch.ones_like(v)
+    v[:, 1::2] = 2.0 ** 127
+    o = swa.swa_prefill(q.to(dev()), k.to(dev()), v.to(dev()), 1)
+    assert torch.equal(o.cpu(), v.repeat_interleave(2, dim=2))
+
+
 # --------------------------------------------------------------- global --
 
 def run_global(B, T, H, Hkv, d, W, g, dtype, seed, rows=None):
@@ -101,18 +114,32 @@ def test_global_f32_small(T, W, g):
 
 
 # ------------------------------------------------------ full workloads --
+# Every head of every sequence at the headline shapes: the rows where the
+# window is still filling or clipped (the first W+128 and the last 128 of a
+# causal sequence; the first and last W/2+128 of a symmetric one), every
+# global row, and at least 1% of the rows drawn at random per head.
 
-def sample_rows(B, Hq, T, W, heads, n_random, seed):
+def head_rows(T, head_start, tail, n_random, rng, extra=()):
+    pick = set(range(min(T, head_start))) | set(range(max(0, T - tail), T)) | set(int(x) for x in extra)
+    mid = np.array(sorted(set(range(T)) - pick))
+    if len(mid):
+        pick |= set(rng.choice(mid, size=min(len(mid), n_random), replace=False).tolist())
+    return np.array(sorted(pick), dtype=np.int64)
+
+
+def all_head_rows(B, H, T, head_start, tail, seed, extra=None):
     rng = np.random.default_rng(seed)
-    rows = []
+    n_random = -(-T // 100)          # at least 1% of the rows of each head
+    bs, hs, is_ = [], [], []
     for b in range(B):
-        for h in heads:
-            pick = set(range(min(T, 130))) | set(range(max(0, T - 130), T))
-            pick |= {x for c in (127, 128, 255, 256, W - 1, W, W + 1, W + 127, W + 128) for x in (c,) if 0 <= x < T}
-            pick |= set(rng.integers(0, T, n_random).tolist())
-            rows += [(b, h, i) for i in sorted(pick)]
-    b, h, i = map(np.array, zip(*rows))
-    return b, h, i
+        for h in range(H):
+            r = head_rows(T, head_start, tail, n_random, rng, extra[b] if extra is not None else ())
+            bs.append(np.full(len(r), b)); hs.append(np.full(len(r), h)); is_.append(r)
+    return np.concatenate(bs), np.concatenate(hs), np.concatenate(is_)
+
+
+def f64(*ts):
+    return [t.double().numpy() for t in ts]
 
 
 def test_tinymistral_full():
@@ -125,35 +152,33 @@ def test_tinymistral_full():
     assert max_err(lse, ref_lse) <= 2e-2
 
 
-def test_mistral_prefill_full_sampled():
+def test_mistral_prefill_full_every_head():
     w = wl.MISTRAL_PREFILL
     inp = wl.make(w)
     lse = torch.empty((w.B, w.Hq, w.T), device=dev())
     o = swa.swa_prefill(inp["q"].to(dev()), inp["k"].to(dev()), inp["v"].to(dev()), w.W, lse=lse)
-    b, h, i = sample_rows(w.B, w.Hq, w.T, w.W, heads=[0, 5, 18, 31], n_random=200, seed=1)
-    ref_o, ref_lse = oracle.swa_prefill(inp["q"], inp["k"], inp["v"], w.W,
-                                        rows=oracle.row_ids(b, h, i, w.Hq, w.T))
-    got = o.cpu()[b, i, h]
-    assert max_err(got, ref_o) <= 2e-2
-    assert max_err(lse.cpu()[b, h, i], ref_lse) <= 2e-2
-    # every row: finite, and rows of one head group share keys only
-    assert torch.isfinite(o).all()
+    o_cpu, lse_cpu = o.cpu(), lse.cpu()
+    assert torch.isfinite(o_cpu).all() and torch.isfinite(lse_cpu).all()
+    b, h, i = all_head_rows(w.B, w.Hq, w.T, w.W + 128, 128, seed=1)
+    assert len(set(h.tolist())) == w.Hq
+    q, k, v = f64(inp["q"], inp["k"], inp["v"])
+    ref_o, ref_lse = oracle.swa_prefill(q, k, v, w.W, rows=oracle.row_ids(b, h, i, w.Hq, w.T))
+    assert max_err(o_cpu[b, i, h], ref_o) <= 2e-2
+    assert max_err(lse_cpu[b, h, i], ref_lse) <= 2e-2
 
 
-def test_longformer_full_sampled():
+def test_longformer_full_every_head():
     w = wl.LONGFORMER
     inp = wl.make(w)
     lse = torch.empty((w.B, w.Hq, w.T), device=dev())
     gi = inp["global_idx"]
     o = swa.swa_prefill_global(inp["q"].to(dev()), inp["k"].to(dev()), inp["v"].to(dev()),
                                gi.to(dev()), w.W, lse=lse)
-    b, h, i = sample_rows(w.B, w.Hq, w.T, w.W // 2, heads=[0, 7, 11], n_random=100, seed=2)
-    # add every global row of the sampled heads
-    extra = [(bb, hh, int(x)) for bb in range(w.B) for hh in (0, 7, 11) for x in gi[bb]]
-    b = np.concatenate([b, [e[0] for e in extra]]); h = np.concatenate([h, [e[1] for e in extra]])
-    i = np.concatenate([i, [e[2] for e in extra]])
-    ref_o, ref_lse = oracle.swa_prefill_global(inp["q"], inp["k"], inp["v"], gi, w.W,
-                                               rows=oracle.row_ids(b, h, i, w.Hq, w.T))
-    assert max_err(o.cpu()[b, i, h], ref_o) <= 2e-2
-    assert max_err(lse.cpu()[b, h, i], ref_lse) <= 2e-2
-    assert torch.isfinite(o).all()
+    o_cpu, lse_cpu = o.cpu(), lse.cpu()
+    assert torch.isfinite(o_cpu).all() and torch.isfinite(lse_cpu).all()
+    b, h, i = all_head_rows(w.B, w.Hq, w.T, w.W // 2 + 128, w.W // 2 + 128, seed=2, extra=gi.numpy())
+    assert len(set(h.tolist())) == w.Hq and len(set(b.tolist())) == w.B
+    q, k, v = f64(inp["q"], inp["k"], inp["v"])
+    ref_o, ref_lse = oracle.swa_prefill_global(q, k, v, gi, w.W, rows=oracle.row_ids(b, h, i, w.Hq, w.T))
+    assert max_err(o_cpu[b, i, h], ref_o) <= 2e-2
+    assert max_err(lse_cpu[b, h, i], ref_lse) <= 2e-2

@@ -7,7 +7,7 @@ import torch
 import decode_swa_prefill_b200 as swa
 import oracle
 from decode_swa_prefill_b200 import workloads as wl
-from gpu_util import dev, max_err
+from gpu_util import dev, max_err, poison_unfilled
 
 pytestmark = pytest.mark.gpu
 
@@ -77,6 +77,9 @@ def test_negative_position_reported():
 
 def run_decode(B, Hq, Hkv, d, W, dtype, seed, lo, hi):
     q, kc, vc, kn, vn, pos = wl.decode_inputs(B, Hq, Hkv, d, W, dtype, seed, lo, hi)
+    # slots past the current token are never written yet: NaN there pins that
+    # the decode never reads them (not merely that it masks them)
+    poison_unfilled(kc, vc, [min(int(p) + 1, W) for p in pos])
     kcd, vcd = kc.to(dev()), vc.to(dev())
     swa.swa_cache_append(kcd, vcd, kn.to(dev()), vn.to(dev()), pos.to(dev()))
     lse = torch.full((B, Hq), float("nan"), device=dev())
@@ -111,8 +114,10 @@ def test_decode_steps_match_prefill_rows_across_wrap():
     qd, kd, vd = q.to(dev()), k.to(dev()), v.to(dev())
     full = swa.swa_prefill(qd, kd, vd, W)
     ref_full, _ = oracle.swa_prefill(q, k, v, W)
-    kc = torch.zeros(B, Hkv, W, d, dtype=torch.bfloat16, device=dev())
-    vc = torch.zeros_like(kc)
+    # the ring starts as NaN: a decode step that read a slot not yet written
+    # would return NaN
+    kc = torch.full((B, Hkv, W, d), float("nan"), dtype=torch.bfloat16, device=dev())
+    vc = torch.full_like(kc, float("nan"))
     worst_vs_prefill = 0.0
     for t in range(T):
         pos = torch.full((B,), t, dtype=torch.int32, device=dev())

@@ -9,7 +9,7 @@ import torch
 import decode_swa_prefill_b200 as swa
 import oracle
 from decode_swa_prefill_b200 import workloads as wl
-from gpu_util import dev, max_err, tol_for
+from gpu_util import dev, max_err, poison_unfilled, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -62,6 +62,10 @@ def test_decode_sinks(dtype, d, Hq, Hkv):
     _, ks, vs, _, _, _ = wl.decode_inputs(B, Hq, Hkv, d, s, dtype, seed=d + Hq + 1, pos_lo=0, pos_hi=1)
     # before any sink left the window, at the edge, long after, wrapped
     pos = torch.tensor([2, 255, 258, 5000, 100000], dtype=torch.int32)
+    # ring slots not written yet, and sink rows the step must take from the
+    # ring instead (sinks still inside the window), are NaN: never read
+    poison_unfilled(kc, vc, [min(int(p) + 1, W) for p in pos])
+    poison_unfilled(ks, vs, [max(0, min(s, int(p) - W + 1)) for p in pos])
     lse = torch.zeros(B, Hq, dtype=torch.float32, device=dev())
     o = swa.swa_decode_sinks(q.to(dev()), kc.to(dev()), vc.to(dev()), ks.to(dev()), vs.to(dev()), pos.to(dev()),
                              lse=lse)
@@ -77,10 +81,11 @@ def test_decode_steps_follow_the_prefill():
     B, T, Hq, Hkv, d, W, s = 1, 300, 8, 2, 128, 64, 4
     q, k, v = wl.prefill_inputs(B, T, Hq, Hkv, d, torch.bfloat16, seed=12)
     ref_o, _ = oracle.swa_prefill_sinks(q, k, v, W, s)
-    kc = torch.zeros(B, Hkv, W, d, dtype=torch.bfloat16, device=dev())
-    vc = torch.zeros_like(kc)
-    ks = torch.zeros(B, Hkv, s, d, dtype=torch.bfloat16, device=dev())
-    vs = torch.zeros_like(ks)
+    # caches start as NaN: a step that read a row not yet written returns NaN
+    kc = torch.full((B, Hkv, W, d), float("nan"), dtype=torch.bfloat16, device=dev())
+    vc = torch.full_like(kc, float("nan"))
+    ks = torch.full((B, Hkv, s, d), float("nan"), dtype=torch.bfloat16, device=dev())
+    vs = torch.full_like(ks, float("nan"))
     qd, kd, vd = q.to(dev()), k.to(dev()), v.to(dev())
     errs = []
     for t in range(T):

@@ -27,7 +27,7 @@ def run(lengths, Hq, Hkv, d, W, dtype, seed):
     q, k, v = q[0], k[0], v[0]
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
     lse = torch.zeros(Hq, total, dtype=torch.float32, device=dev())
-    o = swa.swa_prefill_varlen(q.to(dev()), k.to(dev()), v.to(dev()), cu.to(dev()), W, lse=lse)
+    o = swa.swa_prefill_varlen(q.to(dev()), k.to(dev()), v.to(dev()), cu.to(dev()), W, max(lengths), lse=lse)
     assert swa.swa_get_device_status() == 0
     ref_o, ref_lse = oracle.swa_prefill_varlen(q, k, v, cu, W)
     return o, lse, ref_o, ref_lse
@@ -60,6 +60,6 @@ def test_inconsistent_offsets_reported():
     q, k, v = (t[0].to(dev()) for t in wl.prefill_inputs(1, total, Hq, Hkv, d, torch.bfloat16, 7))
     cu = torch.tensor([0, 60, 40, 100], dtype=torch.int32, device=dev())   # decreasing entry
     assert swa.swa_get_device_status() == 0
-    swa.swa_prefill_varlen(q, k, v, cu, 16, max_seqlen=60)
+    swa.swa_prefill_varlen(q, k, v, cu, 16, 60)
     assert swa.swa_get_device_status() == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_get_device_status() == 0

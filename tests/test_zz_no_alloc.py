@@ -1,38 +1,51 @@
-"""swa_decode_noalloc (scratch in a static device array, for callers that
-cannot allocate device memory) against swa_decode (caller workspace), both
-through the C ABI, on two calls in a row with different inputs.  This file is
-collected last."""
+"""swa_decode_noalloc keeps its split partials in a static device array
+instead of a caller workspace, for callers that cannot allocate device memory
+while they decode.  Checked through the C ABI on two calls in a row with
+different inputs (the array keeps the first call's partials): against the
+fp64 oracle within the decode tolerance, and bit for bit against swa_decode,
+which runs the same kernels with the same split count on a workspace.  Every
+shape here has more than one split, so the static array is really used.
+This file is collected last, so that a failure here leaves every other test
+already run."""
 import pytest
 import torch
 
 import decode_swa_prefill_b200 as swa
+import oracle
 from decode_swa_prefill_b200 import workloads as wl
-from gpu_util import dev, max_err
+from gpu_util import dev, max_err, poison_unfilled, tol_for
 
 pytestmark = pytest.mark.gpu
 
-
-def inputs(w, seed, B=None, W=None):
-    B = B or w.B
-    W = W or w.W
-    q, kc, vc, kn, vn, pos = wl.decode_inputs(B, w.Hq, w.Hkv, w.d, W, w.dtype, seed, w.pos_lo, w.pos_hi)
-    kcd, vcd = kc.to(dev()), vc.to(dev())
-    swa.swa_cache_append(kcd, vcd, kn.to(dev()), vn.to(dev()), pos.to(dev()))
-    return q.to(dev()), kcd, vcd, pos.to(dev())
+# (B, W, dtype, positions drawn from [lo, hi)); split counts 8 and 16
+SHAPES = [
+    (64, 4096, torch.bfloat16, 4096, 131072),   # the 64-sequence decode workload: every slot filled
+    (3, 2048, torch.bfloat16, 0, 3000),         # partly filled rings, other partial offsets
+    (3, 2048, torch.float32, 0, 3000),
+]
 
 
-@pytest.mark.parametrize("B,W", [(64, 4096), (5, 300)])
-def test_noalloc_matches_workspace_decode_twice(B, W):
+@pytest.mark.parametrize("B,W,dtype,lo,hi", SHAPES)
+def test_noalloc_matches_oracle_and_workspace_decode_twice(B, W, dtype, lo, hi):
     w = wl.MISTRAL_DECODE
-    for seed in (101, 202):   # two calls in a row; the scratch keeps the first call's data
-        q, kc, vc, pos = inputs(w, seed, B=B, W=W)
-        lse_ref = torch.empty(B, w.Hq, device=dev())
+    assert swa.swa_decode_workspace_bytes(B, w.Hq, w.Hkv, w.d, W) > 0    # more than one split
+    for seed in (101, 202):   # two calls in a row; the array still holds the first call's partials
+        q, kc, vc, kn, vn, pos = wl.decode_inputs(B, w.Hq, w.Hkv, w.d, W, dtype, seed, lo, hi)
+        poison_unfilled(kc, vc, [min(int(p) + 1, W) for p in pos])
+        kcd, vcd, posd = kc.to(dev()), vc.to(dev()), pos.to(dev())
+        swa.swa_cache_append(kcd, vcd, kn.to(dev()), vn.to(dev()), posd)
+        qd = q.to(dev())
+        lse_ref = torch.full((B, w.Hq), float("nan"), device=dev())
         lse_new = torch.full((B, w.Hq), float("nan"), device=dev())
-        ref = swa.swa_decode(q, kc, vc, pos, lse=lse_ref)
-        got = swa.swa_decode_noalloc(q, kc, vc, pos, lse=lse_new)
+        ref = swa.swa_decode(qd, kcd, vcd, posd, lse=lse_ref)
+        got = swa.swa_decode_noalloc(qd, kcd, vcd, posd, lse=lse_new)
         torch.cuda.synchronize()
-        assert max_err(got, ref.float().cpu().numpy()) <= 2e-2
-        assert max_err(lse_new, lse_ref.cpu().numpy()) <= 2e-2
+        assert torch.equal(got, ref)
+        assert torch.equal(lse_new, lse_ref)
+        rk, rv, _ = oracle.ring_append(kc, vc, kn, vn, pos)
+        ref_o, ref_lse = oracle.swa_decode(q, rk, rv, pos)
+        assert max_err(got, ref_o) <= tol_for(dtype)
+        assert max_err(lse_new, ref_lse) <= max(tol_for(dtype), 1e-5)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
