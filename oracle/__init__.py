@@ -71,6 +71,19 @@ def _load():
         lib.oracle_swa_prefill_dilated.argtypes = [p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
                                                    c_long, c_long, c_int, c_double, p, c_long, c_int]
         lib.oracle_swa_prefill_dilated.restype = c_int
+        lib.oracle_varlen_allowed.argtypes = [c_long, c_long, p, c_long, p]
+        lib.oracle_varlen_allowed.restype = c_int
+        lib.oracle_count_pairs_varlen.argtypes = [p, c_long, p]
+        lib.oracle_count_pairs_varlen.restype = ctypes.c_longlong
+        lib.oracle_swa_prefill_varlen.argtypes = [p, p, p, p, p, p, c_long, p, c_long, c_long, c_long, c_long,
+                                                  c_double, p, c_long, c_int]
+        lib.oracle_swa_prefill_varlen.restype = c_int
+        lib.oracle_paged_append.argtypes = [p, p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long, c_long,
+                                            c_long]
+        lib.oracle_paged_append.restype = c_int
+        lib.oracle_swa_decode_paged.argtypes = [p, p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
+                                                c_long, c_long, c_double]
+        lib.oracle_swa_decode_paged.restype = c_int
         _lib = lib
     return _lib
 
@@ -146,6 +159,45 @@ def ring_append(k_cache, v_cache, k_new, v_new, pos):
     _load().oracle_ring_append(_ptr(kc), _ptr(vc), _ptr(kn), _ptr(vn), _ptr(_i32(pos)), _ptr(slots),
                                B, n, Hkv, d, W)
     return kc, vc, slots
+
+
+def paged_append(k_pages, v_pages, k_new, v_new, pos, page_table):
+    """FIFO append into a paged ring: pools [num_pages,Hkv,P,d], page_table
+    [B,W/P] (ring slot s of sequence b is row s % P of page page_table[b,
+    s // P]); W = P * page_table.shape[1].  Returns (kp, vp, slots) as new
+    fp64 arrays (Ultralytics ring-buffer paragraph; robocikowo.com
+    rolling-buffer entry)."""
+    kp, vp = _f64(k_pages).copy(), _f64(v_pages).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    tbl = _i32(page_table)
+    num_pages, Hkv, P, d = kp.shape
+    B, n = kn.shape[0], kn.shape[1]
+    W = P * tbl.shape[1]
+    slots = np.zeros((B, n), dtype=np.int32)
+    rc = _load().oracle_paged_append(_ptr(kp), _ptr(vp), _ptr(kn), _ptr(vn), _ptr(_i32(pos)), _ptr(tbl),
+                                     _ptr(slots), B, n, Hkv, d, W, P, num_pages)
+    if rc != 0:
+        raise ValueError("page table names a page outside the pool")
+    return kp, vp, slots
+
+
+def swa_decode_paged(q, k_pages, v_pages, page_table, pos, scale=None):
+    """One decode step over a paged ring (layout as paged_append); the
+    current token at pos[b] already appended.  Returns o [B,Hq,d], lse
+    [B,Hq]."""
+    q, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
+    tbl = _i32(page_table)
+    B, Hq, d = q.shape
+    num_pages, Hkv, P = kp.shape[0], kp.shape[1], kp.shape[2]
+    W = P * tbl.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((B, Hq, d)); lse = np.zeros((B, Hq))
+    rc = _load().oracle_swa_decode_paged(_ptr(q), _ptr(kp), _ptr(vp), _ptr(tbl), _ptr(_i32(pos)), _ptr(o),
+                                         _ptr(lse), B, Hq, Hkv, d, W, P, num_pages, float(scale))
+    if rc != 0:
+        raise ValueError("negative position or a page outside the pool")
+    return o, lse
 
 
 # ---------------------------------------------------------------- prefill --
@@ -316,21 +368,54 @@ def swa_prefill_dilated(q, k, v, W, dil, mode=CAUSAL, scale=None, rows=None, nth
 
 # ----------------------------------------------------------------- varlen --
 
-def swa_prefill_varlen(q, k, v, cu_seqlens, W, scale=None, nthreads=None):
+def _windows(W, nseq):
+    """One window per sequence: W is an int (every sequence) or a sequence of
+    nseq ints."""
+    if np.ndim(W) == 0:
+        return np.full(nseq, int(W), dtype=np.int32)
+    w = _i32(W).reshape(-1)
+    assert len(w) == nseq, "one window per sequence"
+    return w
+
+
+def varlen_allowed(r, j, cu_seqlens, W):
+    """Packed rows: row r sees row j of its own sequence with r-W_s+1 <= j <= r
+    (robocikowo.com opening definition, per sequence)."""
+    cu = _i32(cu_seqlens)
+    return bool(_load().oracle_varlen_allowed(r, j, _ptr(cu), len(cu) - 1, _ptr(_windows(W, len(cu) - 1))))
+
+
+def count_pairs_varlen(cu_seqlens, W):
+    cu = _i32(cu_seqlens)
+    return int(_load().oracle_count_pairs_varlen(_ptr(cu), len(cu) - 1, _ptr(_windows(W, len(cu) - 1))))
+
+
+def swa_prefill_varlen(q, k, v, cu_seqlens, W, scale=None, rows=None, nthreads=None):
     """Causal window over packed sequences: q [total,Hq,d], k/v
-    [total,Hkv,d]; sequence b holds rows cu_seqlens[b] .. cu_seqlens[b+1]-1
-    and attends within itself only (every sequence is its own causal
-    prefill, robocikowo.com opening definition).  Returns o [total,Hq,d] and
-    lse [Hq,total]."""
+    [total,Hkv,d]; sequence s holds rows cu_seqlens[s] .. cu_seqlens[s+1]-1
+    and attends within itself only, with its own window W[s] (W an int: the
+    same window for all).  Every sequence is its own causal prefill
+    (robocikowo.com opening definition); the windows may differ as between
+    the local layers of different models (Ultralytics glossary, section on
+    alternating local and global layers).  rows=None returns o [total,Hq,d]
+    and lse [Hq,total]; otherwise rows are flattened h*total + r ids and the
+    result is o [nrows,d], lse [nrows]."""
     q, k, v = _f64(q), _f64(k), _f64(v)
-    cu = [int(x) for x in _i32(cu_seqlens)]
+    cu = _i32(cu_seqlens)
+    nseq = len(cu) - 1
     total, Hq, d = q.shape
-    o = np.zeros((total, Hq, d)); lse = np.zeros((Hq, total))
-    for b in range(len(cu) - 1):
-        lo, hi = cu[b], cu[b + 1]
-        if hi <= lo:
-            continue
-        ob, lb = swa_prefill(q[None, lo:hi], k[None, lo:hi], v[None, lo:hi], W, scale=scale, nthreads=nthreads)
-        o[lo:hi] = ob[0]
-        lse[:, lo:hi] = lb[0]
-    return o, lse
+    Hkv = k.shape[1]
+    w = _windows(W, nseq)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r = _rows_arg(rows, 1, Hq, total)
+    o = np.zeros((len(r), d)); lse = np.zeros(len(r))
+    rc = _load().oracle_swa_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu), nseq, _ptr(w),
+                                           total, Hq, Hkv, d, float(scale), _ptr(r), len(r),
+                                           nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("inconsistent offsets or a window below 1")
+    if rows is not None:
+        return o, lse
+    o, lse = _unflatten(o, lse, r, True, 1, total, Hq, d)
+    return o[0], lse[0]

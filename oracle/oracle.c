@@ -38,6 +38,7 @@
 #define ORACLE_CAUSAL 0
 #define ORACLE_SYMMETRIC 1
 #define ORACLE_SINKS 2
+#define ORACLE_VARLEN 3
 
 /* ---------------------------------------------------------------- masks -- */
 
@@ -78,6 +79,33 @@ int oracle_sink_allowed(long i, long j, long T, long W, long s)
 {
     if (j < 0 || j >= T || i < 0 || i >= T || j > i) return 0;
     return j >= i - W + 1 || j < s;
+}
+
+/* Packed variable-length batch, one causal window per sequence [P3 opening
+ * definition: query i sees keys i-W+1 .. i; P4 section on alternating local
+ * and global layers: Gemma 2 used a 4,096-token window and Gemma 3 a
+ * 1,024-token one, so one batch may hold sequences whose windows differ].
+ * Packed rows cu[s] .. cu[s+1]-1 hold sequence s.  Row r of sequence s sees
+ * packed row j when j belongs to the same sequence and r - wseq[s] + 1 <= j
+ * <= r.  A row outside every sequence sees nothing. */
+int oracle_varlen_allowed(long r, long j, const int32_t *cu, long nseq, const int32_t *wseq)
+{
+    for (long s = 0; s < nseq; s++) {
+        if (r < cu[s] || r >= cu[s + 1]) continue;
+        if (j < cu[s] || j >= cu[s + 1]) return 0;
+        return j <= r && j >= r - (long)wseq[s] + 1;
+    }
+    return 0;
+}
+
+/* Pairs the packed batch allows, counted cell by cell over [total,total]. */
+long long oracle_count_pairs_varlen(const int32_t *cu, long nseq, const int32_t *wseq)
+{
+    const long total = nseq > 0 ? cu[nseq] : 0;
+    long long n = 0;
+    for (long r = 0; r < total; r++)
+        for (long j = 0; j < total; j++) n += oracle_varlen_allowed(r, j, cu, nseq, wseq);
+    return n;
 }
 
 /* Dilated window [P2 s.4.2: instead of all W neighbours, every dil-th token
@@ -187,6 +215,47 @@ void oracle_ring_append(double *kc, double *vc, const double *kn, const double *
         }
 }
 
+/* Paged ring: the W slots of a sequence's ring live in W/P pages of P slots
+ * taken from a shared pool, in any order [P4 ring-buffer paragraph: position
+ * i goes to slot i mod w, overwriting the oldest entry; P5 check-yourself
+ * question 1: the cache holds only the window, so a sequence never needs more
+ * than W slots].  Pool [num_pages,Hkv,P,d]; table [B, W/P]: ring slot s of
+ * sequence b is row s mod P of page table[b, s / P].  Returns the address of
+ * that row for kv head h, or NULL when the table names no page of the pool. */
+static double *paged_row(double *pool, const int32_t *table, long b, long h, long s, long Hkv, long d, long W,
+                         long P, long num_pages)
+{
+    const long page = table[b * (W / P) + s / P];
+    if (page < 0 || page >= num_pages) return NULL;
+    return pool + ((page * Hkv + h) * P + s % P) * d;
+}
+
+/* Append into a paged ring: token t of sequence b (position pos[b]+t) goes to
+ * ring slot (pos[b]+t) mod W, i.e. into its page as paged_row says; tokens
+ * are written one after the other, oldest first (FIFO overwrite) [P3
+ * rolling-buffer entry].  Returns -1 if a slot's page is outside the pool
+ * (nothing is written for that token). */
+int oracle_paged_append(double *kp, double *vp, const double *kn, const double *vn, const int32_t *pos,
+                        const int32_t *table, int32_t *slot_out, long B, long n, long Hkv, long d, long W, long P,
+                        long num_pages)
+{
+    int rc = 0;
+    for (long b = 0; b < B; b++)
+        for (long t = 0; t < n; t++) {
+            const long s = oracle_slot((long)pos[b] + t, W);
+            if (slot_out) slot_out[b * n + t] = (int32_t)s;
+            for (long h = 0; h < Hkv; h++) {
+                double *kd = paged_row(kp, table, b, h, s, Hkv, d, W, P, num_pages);
+                double *vd = paged_row(vp, table, b, h, s, Hkv, d, W, P, num_pages);
+                if (!kd || !vd) { rc = -1; continue; }
+                const double *ksrc = kn + ((b * n + t) * Hkv + h) * d;
+                const double *vsrc = vn + ((b * n + t) * Hkv + h) * d;
+                for (long e = 0; e < d; e++) { kd[e] = ksrc[e]; vd[e] = vsrc[e]; }
+            }
+        }
+    return rc;
+}
+
 /* ------------------------------------------------------ one attention row -- */
 
 /* Softmax-weighted sum over an explicit key list [P2 s.9: scores, forbidden
@@ -232,6 +301,9 @@ typedef struct {
     long nrows;
     long next;           /* work counter */
     pthread_mutex_t mu;
+    const int32_t *cu;   /* packed sequences (mode ORACLE_VARLEN): offsets [nseq+1] */
+    long nseq;
+    const int32_t *wseq; /* window of each sequence [nseq] */
 } prefill_job;
 
 static void prefill_one(prefill_job *J, long r, const double **kr, const double **vr, double *s)
@@ -246,6 +318,7 @@ static void prefill_one(prefill_job *J, long r, const double **kr, const double 
     for (long j = 0; j < J->T; j++) {
         int ok;
         if (J->mode == ORACLE_SINKS) ok = oracle_sink_allowed(i, j, J->T, J->W, J->sinks);
+        else if (J->mode == ORACLE_VARLEN) ok = oracle_varlen_allowed(i, j, J->cu, J->nseq, J->wseq);
         else if (J->dil > 1) ok = oracle_dilated_allowed(i, j, J->T, J->W, J->dil, J->mode);
         else ok = oracle_allowed(i, j, J->T, J->W, J->mode, gb, gb ? J->g : 0);
         if (!ok) continue;
@@ -335,6 +408,23 @@ int oracle_swa_prefill_dilated(const double *q, const double *k, const double *v
     return run_prefill(&J, nthreads);
 }
 
+/* Packed variable-length prefill with one window per sequence (see
+ * oracle_varlen_allowed): q, o [total,Hq,d]; k, v [total,Hkv,d]; rows are
+ * flattened h*total + r; o [nrows,d], lse (nullable) [nrows]. */
+int oracle_swa_prefill_varlen(const double *q, const double *k, const double *v, double *o, double *lse,
+                              const int32_t *cu, long nseq, const int32_t *wseq, long total, long Hq, long Hkv,
+                              long d, double scale, const int64_t *rows, long nrows, int nthreads)
+{
+    if (nseq < 0 || (nseq > 0 && cu[nseq] != total)) return -1;
+    for (long s = 0; s < nseq; s++)
+        if (cu[s] > cu[s + 1] || wseq[s] < 1) return -1;
+    prefill_job J = {q, k, v, o, lse, 1, total, Hq, Hkv, d, 0, ORACLE_VARLEN, NULL, 0, 0, 1, scale, rows, nrows};
+    J.cu = cu;
+    J.nseq = nseq;
+    J.wseq = wseq;
+    return run_prefill(&J, nthreads);
+}
+
 /* ----------------------------------------------------------------- decode -- */
 
 /* One decode step over the ring cache [P4 ring-buffer paragraph; P5
@@ -365,6 +455,40 @@ int oracle_swa_decode(const double *q, const double *kc, const double *vc, const
     }
     free(kr); free(vr); free(s);
     return 0;
+}
+
+/* One decode step over a paged ring (see paged_row): the current token at
+ * position pos[b] is already appended; the visible keys are ring slots
+ * 0 .. min(pos+1,W)-1, in slot order, each read through the page table [P4
+ * ring-buffer paragraph].  Returns -1 for a negative position or a page
+ * outside the pool. */
+int oracle_swa_decode_paged(const double *q, const double *kp, const double *vp, const int32_t *table,
+                            const int32_t *pos, double *o, double *lse, long B, long Hq, long Hkv, long d, long W,
+                            long P, long num_pages, double scale)
+{
+    for (long b = 0; b < B; b++)
+        if (pos[b] < 0) return -1;
+    const double **kr = malloc(sizeof(double *) * (size_t)W);
+    const double **vr = malloc(sizeof(double *) * (size_t)W);
+    double *sc = malloc(sizeof(double) * (size_t)W);
+    int rc = 0;
+    for (long b = 0; b < B && rc == 0; b++) {
+        const long nvalid = (long)pos[b] + 1 < W ? (long)pos[b] + 1 : W;
+        for (long h = 0; h < Hq && rc == 0; h++) {
+            const long hk = h * Hkv / Hq;
+            for (long sl = 0; sl < nvalid; sl++) {
+                kr[sl] = paged_row((double *)kp, table, b, hk, sl, Hkv, d, W, P, num_pages);
+                vr[sl] = paged_row((double *)vp, table, b, hk, sl, Hkv, d, W, P, num_pages);
+                if (!kr[sl] || !vr[sl]) rc = -1;
+            }
+            if (rc) break;
+            double l;
+            attend_row(q + (b * Hq + h) * d, kr, vr, nvalid, d, scale, o + (b * Hq + h) * d, &l, sc);
+            if (lse) lse[b * Hq + h] = l;
+        }
+    }
+    free(kr); free(vr); free(sc);
+    return rc;
 }
 
 /* ---------------------------------------------------------- chunk prefill -- */
