@@ -314,6 +314,7 @@ def gpu_arm(args, world, rank, local):
     sinks = sinks_arm(swa, dev, args, load_peaks()[0])
     dilated = dilated_arm(swa, dev, args, load_peaks()[0])
     varlen = varlen_arm(swa, dev, args, load_peaks()[0])
+    paged = paged_arm(swa, st, dev, args, load_peaks()[0])
 
     peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
@@ -347,6 +348,7 @@ def gpu_arm(args, world, rank, local):
             "sinks": sinks,
             "dilated": dilated,
             "varlen": varlen,
+            "paged_decode": paged,
             "decode": {"gbs": round(dec_gbs, 1), "us": round(avg["decode"] * 1e3, 2),
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
@@ -510,8 +512,62 @@ def varlen_arm(swa, dev, args, peaks):
             times.append(e0.elapsed_time(e1))
     ms = sum(times) / len(times)
     tf = flops / (ms * 1e-3) / 1e12
-    return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
-            "flops": flops, "lengths": lengths}
+    res = {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+           "flops": flops, "lengths": lengths}
+    # the same batch with one window per sequence: 1,024 and 4,096 tokens
+    # alternating (the local-layer windows of Gemma 3 and Gemma 2)
+    windows = [1024 if s % 2 == 0 else 4096 for s in range(len(lengths))]
+    win = torch.tensor(windows, dtype=torch.int32, device=dev)
+    flops_m = sum(causal_pairs(n, W) for n, W in zip(lengths, windows)) * w.Hq * 4 * w.d
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill_varlen(q, k, v, cu, win, max(lengths), o=o)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    tf = flops_m / (ms * 1e-3) / 1e12
+    res["mixed_windows"] = {"windows": windows, "tflops": round(tf, 2), "ms": round(ms, 4),
+                            "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "flops": flops_m}
+    return res
+
+
+def paged_arm(swa, st, dev, args, peaks):
+    """Decode over a paged ring: the 64-sequence decode workload with each
+    ring split into pages of 16 slots scattered over a shared pool in a
+    seeded random order; not part of the step.  Bytes are the K/V rows read,
+    as for the dense decode."""
+    D, P = wl.MISTRAL_DECODE, 16
+    npg = D.W // P
+    g = torch.Generator().manual_seed(77)
+    table = torch.randperm(D.B * npg, generator=g).reshape(D.B, npg).to(torch.int32).to(dev)
+    kp = torch.empty(D.B * npg, D.Hkv, P, D.d, dtype=D.dtype, device=dev)
+    vp = torch.empty_like(kp)
+    s = torch.arange(D.W, device=dev)
+    for b in range(D.B):
+        kp[table[b, s // P].long(), :, s % P] = st.kc[b].permute(1, 0, 2)
+        vp[table[b, s // P].long(), :, s % P] = st.vc[b].permute(1, 0, 2)
+    o = torch.empty_like(st.dq)
+    nbytes = D.B * D.Hkv * D.W * D.d * 2 * 2
+    times = []
+    for i in range(args.warmup + max(10, args.steps // 2)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_decode_paged(st.dq, kp, vp, table, st.pos, o=o, workspace=st.ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = sum(times) / len(times)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    same = bool(torch.equal(o, st.do))
+    del kp, vp
+    return {"page_size": P, "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+            "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
+            "equal_to_dense_decode": same}
 
 
 def sink_pairs(T, W, s):

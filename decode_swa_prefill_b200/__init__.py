@@ -8,6 +8,10 @@ libswa.so is missing or cannot be loaded, every call raises.
 
 Layouts: q/o [B,T,Hq,d], k/v [B,T,Hkv,d], lse [B,Hq,T] (fp32), ring caches
 [B,Hkv,W,d], decode q/o [B,Hq,d], positions int32.
+
+With the environment variable SWA_DEBUG=1 the debug build libswa_debug.so is
+loaded instead: the same kernels with device-side checks of their tile, row
+and slot indices, reported as SWA_ERR_INTERNAL by swa_get_device_status.
 """
 import ctypes
 import os
@@ -21,12 +25,15 @@ __all__ = [
     "swa_decode_sinks",
     "swa_decode_workspace_bytes", "swa_mask_export", "swa_get_device_status",
     "swa_debug_expire_wait", "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
+    "swa_cache_append_paged", "swa_decode_paged",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libswa.so")
+DEBUG = os.environ.get("SWA_DEBUG", "0") not in ("", "0")
+library_path = os.path.join(_HERE, "libswa_debug.so" if DEBUG else "libswa.so")
 
 SWA_OK, SWA_ERR_INVALID_ARG, SWA_ERR_UNSUPPORTED, SWA_ERR_CUDA, SWA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SWA_ERR_INTERNAL = 5
 SWA_DTYPE_F32, SWA_DTYPE_BF16 = 0, 1
 
 # every symbol include/swa.h declares
@@ -35,7 +42,8 @@ EXPORTED = [
     "swa_prefill_dilated", "swa_prefill_dilated_workspace_bytes", "swa_prefill_varlen",
     "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
-    "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc",
+    "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc", "swa_cache_append_paged",
+    "swa_decode_paged",
 ]
 
 _lib = None
@@ -53,8 +61,8 @@ def load():
     if _lib is not None:
         return _lib
     if not os.path.exists(library_path):
-        raise RuntimeError("libswa.so not found at %s; build it with "
-                           "`python -m decode_swa_prefill_b200.build`" % library_path)
+        raise RuntimeError("%s not found; build it with `python -m decode_swa_prefill_b200.build%s`"
+                           % (library_path, " --debug" if DEBUG else ""))
     lib = ctypes.CDLL(library_path)
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.swa_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P]
@@ -64,13 +72,15 @@ def load():
     lib.swa_prefill_dilated.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_prefill_dilated_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
     lib.swa_prefill_dilated_workspace_bytes.restype = ctypes.c_size_t
-    lib.swa_prefill_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+    lib.swa_prefill_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P]
     lib.swa_decode_sinks.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_cache_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.swa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.swa_cache_append_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+    lib.swa_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
     lib.swa_mask_export.argtypes = [P, I, I, I, P, I, P]
     lib.swa_get_device_status.argtypes = [P]
     lib.swa_debug_expire_wait.argtypes = [I, P]
@@ -81,7 +91,8 @@ def load():
     for name in ("swa_prefill", "swa_prefill_global", "swa_prefill_chunk", "swa_prefill_sinks", "swa_decode_sinks",
                  "swa_prefill_dilated", "swa_prefill_varlen",
                  "swa_cache_append", "swa_decode",
-                 "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait"):
+                 "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
+                 "swa_cache_append_paged", "swa_decode_paged"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -143,18 +154,24 @@ def swa_prefill(q, k, v, W, scale=None, o=None, lse=None, stream=None):
 def swa_prefill_varlen(q, k, v, cu_seqlens, W, max_seqlen, scale=None, o=None, lse=None, stream=None):
     """Causal window over packed sequences q [total,Hq,d], k/v [total,Hkv,d];
     cu_seqlens int32 [nseq+1] on the device; max_seqlen is the longest
-    sequence (a host integer the caller knows, like the offsets themselves)."""
-    _dev_contig(q, k, v, o, lse, cu_seqlens)
+    sequence (a host integer the caller knows, like the offsets themselves).
+    W is one window for every sequence (int) or one per sequence (int32
+    tensor [nseq] on the device)."""
+    windows = W if isinstance(W, torch.Tensor) else None
+    _dev_contig(q, k, v, o, lse, cu_seqlens, windows)
     total, Hq, d = q.shape
     Hkv = k.shape[1]
     _need(k.shape == (total, Hkv, d) and v.shape == k.shape, "k/v shape")
     _need(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1, "cu_seqlens int32 [nseq+1]")
     nseq = cu_seqlens.numel() - 1
+    if windows is not None:
+        _need(windows.dtype == torch.int32 and windows.shape == (nseq,), "windows int32 [nseq]")
     if o is None:
         o = torch.empty_like(q)
     scale = d ** -0.5 if scale is None else scale
-    st = load().swa_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), nseq, total,
-                                   int(max_seqlen), Hq, Hkv, d, W, float(scale), _dtype_code(q), _stream(stream))
+    st = load().swa_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), _ptr(windows),
+                                   nseq, total, int(max_seqlen), Hq, Hkv, d, 1 if windows is not None else int(W),
+                                   float(scale), _dtype_code(q), _stream(stream))
     _check(st, "swa_prefill_varlen")
     return o
 
@@ -251,6 +268,47 @@ def swa_cache_append(k_cache, v_cache, k_new, v_new, pos, slot_out=None, stream=
     st = load().swa_cache_append(_ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(pos),
                                  _ptr(slot_out), B, n, Hkv, d, W, _dtype_code(k_cache), _stream(stream))
     _check(st, "swa_cache_append")
+
+
+def swa_cache_append_paged(k_pages, v_pages, k_new, v_new, pos, page_table, slot_out=None, stream=None):
+    """Write k_new/v_new [B,n,Hkv,d] into ring slots (pos[b]+t) mod W of a
+    paged ring: pools [num_pages,Hkv,P,d], page_table int32 [B, W/P]."""
+    _dev_contig(k_pages, v_pages, k_new, v_new, pos, page_table, slot_out)
+    num_pages, Hkv, P, d = k_pages.shape
+    B, n = k_new.shape[0], k_new.shape[1]
+    _need(k_new.shape == (B, n, Hkv, d) and v_new.shape == k_new.shape, "k_new/v_new shape")
+    _need(v_pages.shape == k_pages.shape, "pool shape")
+    _need(page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.shape[0] == B, "page_table")
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    W = P * page_table.shape[1]
+    st = load().swa_cache_append_paged(_ptr(k_pages), _ptr(v_pages), _ptr(k_new), _ptr(v_new), _ptr(pos),
+                                       _ptr(page_table), _ptr(slot_out), B, n, Hkv, d, W, P, num_pages,
+                                       _dtype_code(k_pages), _stream(stream))
+    _check(st, "swa_cache_append_paged")
+
+
+def swa_decode_paged(q, k_pages, v_pages, page_table, pos, scale=None, o=None, lse=None, workspace=None,
+                     stream=None):
+    """One decode step over a paged ring (pools [num_pages,Hkv,P,d],
+    page_table int32 [B, W/P]); pos[b] already appended."""
+    _dev_contig(q, k_pages, v_pages, page_table, pos, o, lse, workspace)
+    B, Hq, d = q.shape
+    num_pages, Hkv, P = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    _need(page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.shape[0] == B, "page_table")
+    _need(pos.dtype == torch.int32 and pos.numel() == B, "pos [B] int32")
+    W = P * page_table.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    need = swa_decode_workspace_bytes(B, Hq, Hkv, d, W)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(o), _ptr(lse),
+                                 _ptr(pos), B, Hq, Hkv, d, W, P, num_pages, float(scale), _dtype_code(q),
+                                 _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "swa_decode_paged")
+    return o
 
 
 def swa_decode_workspace_bytes(B, Hq, Hkv, d, W):

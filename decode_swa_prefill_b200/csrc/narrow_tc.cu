@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(NB_THREADS, 1)
         int jq = 0, it = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++it) {
             const NUnit x = nb_unit(u, n_kp, nqt, n_slice, G);
+            SWA_DCHECK(x.q0 >= 0 && x.q0 < a.T && x.kp < n_kp && x.h0 + G <= a.Hq, a.ctl.status);
             const int ks = it % C::KVST;
             ok = warp_wait_bounded(&bars->kv_empty[ks], ((it / C::KVST) & 1) ^ 1, ctl);
             if (!ok) break;

@@ -1,0 +1,619 @@
+// Sliding-window prefill on tcgen05 tensor cores with 128-key tiles and two
+// query tiles in alternation (sm_100a).
+//
+// What it computes (the pages' definition): for query row i, softmax over the
+// keys of its window of scale*q.k, logits outside the window being -inf, then
+// the weighted sum of value rows ("Sliding Window Attention", robocikowo.com,
+// opening definition).  The [T,T] score matrix never exists: a CTA streams
+// only the 128-key tiles that intersect its query tiles' windows (the
+// fused-kernel point of the same page and of the Ultralytics glossary's
+// FlashAttention entry); work per query tile is O(W*d).
+//
+// CTA anatomy (320 threads, one CTA per SM), two 128-row query tiles X = A, B
+// sharing one kv head, hence every K/V tile: the two query heads of a GQA pair
+// at the same rows, or (odd group size) two consecutive row tiles of one head.
+//   warps 0-3  softmax + epilogue of tile A: thread r owns row r = TMEM lane r
+//   warps 4-7  the same for tile B
+//   warp 8     producer: TMA tile loads of Q (once), K and V (128 keys per
+//              tile, two stages each); no multicast
+//   warp 9     TMEM allocator and the single MMA issuer (lane 0)
+// TMEM (all 512 columns):
+//   S[X]  columns 128X .. 128X+127: fp32 scores of one 128-key tile
+//   P[X]  the first 64 columns of S[X]: bf16 probabilities (pairs)
+//   O[X]  columns 256+128X: fp32 output accumulator (d <= 128)
+// Per key tile t the issuer runs, in this order,
+//   PV_A(t-1), QK_A(t), PV_B(t-1), QK_B(t)
+// (PV_X: O[X] += P[X] V, A operand from TMEM; QK_X: S[X] = Q_X K^T), so the
+// softmax of one tile runs while the tensor core computes the other tile's
+// PV and next QK^T.  QK_X(t) overwrites the S[X] columns that PV_X(t-1) reads
+// P from; both come from the one issuing thread, and the tensor core executes
+// one thread's tcgen05.mma operations in issue order, so no wait separates
+// them.  With 128-key tiles every QK^T has N = 128: both operands come from
+// shared memory at the rate the tensor core consumes them (an N = 64 QK^T is
+// limited by shared-memory bandwidth instead).
+//
+// Softmax (one row per thread, 128 scores per tile): running maximum in log2
+// units, raised only when a tile's maximum exceeds it by more than 2^8 (P
+// stays <= 256 in bf16), which rescales l and the O row in TMEM after the
+// previous PV; -inf outside the window on edge tiles only; per warp, 32-key
+// chunks no row of the warp can see are skipped (their P is written as 0).
+// Three quarters of the exponentials run on the MUFU (ex2.approx), one
+// quarter as the range-reduced cubic exp2_poly2 on the FMA pipe.
+//
+// Every mbarrier wait is bounded (wait_bounded): on expiry the CTA records
+// SWA_STATUS_TIMEOUT, drains its own in-flight copies and MMAs with a second
+// bound, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "ptx.cuh"
+#include "swa_internal.h"
+#include "tma_map.h"
+
+namespace swa {
+namespace {
+
+constexpr int PP_BM = 128;               // query rows per tile (= TMEM lanes)
+constexpr int PP_BN = 128;               // keys per key tile
+constexpr int PP_NSTAGE = 2;             // K and V pipeline depth
+constexpr int PP_THREADS = 320;
+constexpr float PP_RESCALE_LOG2 = 8.0f;  // raise the running max only beyond 2^8
+constexpr int PP_POLY_EVERY = 4;         // every 4th pair of exponentials on the FMA pipe
+
+template <int D>
+struct PCfg {
+    static constexpr int RB = (D * 2 >= 128) ? 128 : D * 2; // bytes per swizzled row
+    static constexpr int E = RB / 2;                         // elements per chunk row
+    static constexpr int NCH = D / E;                        // chunks per head row
+    static constexpr int QCH = PP_BM * RB;                   // one chunk of a 128-row Q tile
+    static constexpr int KCH = PP_BN * RB;                   // one chunk of a 128-key tile
+    static constexpr int QTILE = PP_BM * D * 2;
+    static constexpr int KTILE = PP_BN * D * 2;
+    static constexpr uint32_t LAYOUT = (RB == 128) ? UMMA_SW128 : UMMA_SW64;
+    static constexpr int OFF_Q = 0;                          // Q_A, Q_B
+    static constexpr int OFF_K = OFF_Q + 2 * QTILE;
+    static constexpr int OFF_V = OFF_K + PP_NSTAGE * KTILE;
+    static constexpr int OFF_BAR = OFF_V + PP_NSTAGE * KTILE;
+    // + room to align the base to 1 KiB; more than half the SM's shared
+    // memory so that a second CTA never shares the SM (each CTA takes all
+    // 512 TMEM columns)
+    static constexpr int SMEM_NEED = OFF_BAR + 256 + 1024;
+    static constexpr int SMEM_BYTES = SMEM_NEED > 120 * 1024 ? SMEM_NEED : 120 * 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(D == 32 || D == 64 || D == 128, "head dim");
+    static_assert(SMEM_BYTES + 1024 <= 228 * 1024, "fits one SM");
+    static_assert(2 * (SMEM_BYTES + 1024) > 228 * 1024, "never two CTAs per SM");
+};
+
+__host__ __device__ constexpr uint32_t pp_col_s(int x) { return 128u * x; }
+__host__ __device__ constexpr uint32_t pp_col_o(int x) { return 256u + 128u * x; }
+
+// Byte offset of element e of row r inside a swizzled [rows][D] tile whose
+// E-element chunks are `ch_bytes` apart (the layout of a TMA SWIZZLE_128B /
+// SWIZZLE_64B load).
+template <int D>
+__device__ __forceinline__ uint32_t pp_tile_offset(int r, int e, int ch_bytes)
+{
+    using C = PCfg<D>;
+    const int ch = e / C::E;
+    const int u = (e % C::E) / 8;
+    const int phys = (C::RB == 128) ? (u ^ (r & 7)) : (u ^ ((r >> 1) & 3));
+    return ch * ch_bytes + r * C::RB + phys * 16;
+}
+
+struct PPBars {
+    uint64_t q_full;
+    uint64_t k_full[PP_NSTAGE];
+    uint64_t k_empty[PP_NSTAGE];
+    uint64_t v_full[PP_NSTAGE];
+    uint64_t v_empty[PP_NSTAGE];
+    uint64_t s_full[2];    // [tile]
+    uint64_t p_full[2];    // [tile], one arrival per softmax warp
+    uint64_t pv_done[2];   // [tile]
+    uint64_t epi[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ void pp_drain_wait(uint64_t *bar, uint32_t parity, unsigned long long limit)
+{
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > limit) return;
+    }
+}
+
+// One 128-row query tile of a CTA: key tiles [ts, te) relative to j_lo.
+struct PPTile {
+    int h, m0, nrows, ts, te;
+    bool active;
+};
+
+struct PPWork {
+    int b, hk;
+    PPTile q[2];
+    int j_lo;      // first key tile (absolute, 128-key units)
+    int n_tiles;   // key tiles the CTA streams
+};
+
+__device__ __forceinline__ bool pp_active(const PPTile &q, int t) { return q.active && t >= q.ts && t < q.te; }
+
+// Units: pairs of query heads of one kv head (even group size) or pairs of
+// consecutive row tiles of one head; query tiles in descending order, so the
+// short CTAs at the start of a causal sequence run last and fill the tail.
+__device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a)
+{
+    PPWork w;
+    const int G = a.Hq / a.Hkv;
+    const int nqt = (a.T + PP_BM - 1) / PP_BM;
+    const int bid = blockIdx.x;
+    for (int x = 0; x < 2; ++x) w.q[x] = PPTile{0, 0, 0, 0, 0, false};
+    if (G % 2 == 0) {
+        const int hp = bid % (a.Hq / 2);
+        const int qt = nqt - 1 - (bid / (a.Hq / 2)) % nqt;
+        w.b = bid / ((a.Hq / 2) * nqt);
+        for (int x = 0; x < 2; ++x) w.q[x] = PPTile{2 * hp + x, qt * PP_BM, min(PP_BM, a.T - qt * PP_BM), 0, 0, true};
+    } else {
+        const int h = bid % a.Hq;
+        const int nqp = (nqt + 1) / 2;
+        const int qp = nqp - 1 - (bid / a.Hq) % nqp;
+        w.b = bid / (a.Hq * nqp);
+        for (int x = 0; x < 2; ++x) {
+            const int qt = 2 * qp + x;
+            if (qt < nqt) w.q[x] = PPTile{h, qt * PP_BM, min(PP_BM, a.T - qt * PP_BM), 0, 0, true};
+        }
+    }
+    int lo = a.T, hi = -1;
+    int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+    for (int x = 0; x < 2; ++x) {
+        if (!w.q[x].active) continue;
+        lo_x[x] = max(0, w.q[x].m0 - a.left);
+        hi_x[x] = min(a.T - 1, w.q[x].m0 + PP_BM - 1 + a.right);
+        lo = min(lo, lo_x[x]);
+        hi = max(hi, hi_x[x]);
+    }
+    w.j_lo = lo / PP_BN;
+    w.n_tiles = hi / PP_BN - w.j_lo + 1;
+    for (int x = 0; x < 2; ++x)
+        if (w.q[x].active) {
+            w.q[x].ts = lo_x[x] / PP_BN - w.j_lo;
+            w.q[x].te = hi_x[x] / PP_BN - w.j_lo + 1;
+        }
+    w.hk = w.q[0].h / G;
+    return w;
+}
+
+// Softmax of one 128-key tile for one row: scores -> running max / sum -> P
+// (bf16 pairs) over the first 64 columns of the tile's S columns, in two
+// passes over TMEM so that at most 64 scores are held in registers: the row
+// maximum from two 64-column halves, then per 32-column chunk the scores
+// again, their exponentials and the chunk's 16 columns of P.  P of chunk cc
+// lands in columns 16cc .. 16cc+15, which belong to S chunks already read
+// (cc/2 <= cc), so no score is overwritten before it is used.  FULL: every key
+// of the tile is visible to every row of the warp (no masking, all chunks
+// live), the common case, compiled without the masking branches.
+template <bool FULL>
+__device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c_hi, int col_lo, int col_hi,
+                                                float scale_log2, float &m, float &l, bool &rescale, float &alpha,
+                                                bool first)
+{
+    auto live = [&](int cc) { return FULL || (cc >= c_lo && cc <= c_hi); };
+    auto mask32 = [&](float *v, int cc) {
+        if (!FULL) {
+            if (!live(cc)) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = -CUDART_INF_F;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int xx = cc * 32 + e;
+                    if (xx < col_lo || xx > col_hi) v[e] = -CUDART_INF_F;
+                }
+            }
+        }
+    };
+    // ---- pass 1: row maximum ----
+    float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float sr[64];
+        if (live(2 * hh)) tmem_ld32(s_addr + hh * 64, sr);
+        if (live(2 * hh + 1)) tmem_ld32(s_addr + hh * 64 + 32, sr + 32);
+        tmem_ld_wait_dep(sr);
+        reg_fence32(sr + 32);
+        mask32(sr, 2 * hh);
+        mask32(sr + 32, 2 * hh + 1);
+#pragma unroll
+        for (int e = 0; e + 8 <= 64; e += 8)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], sr[e + j], sr[e + 4 + j]);
+    }
+    const float mt = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
+    rescale = false;
+    alpha = 1.f;
+    if (mt > m + PP_RESCALE_LOG2) {
+        alpha = ex2_approx(m - mt);     // 0 when m was -inf
+        l *= alpha;
+        rescale = !first;
+        m = mt;
+    }
+    // ---- pass 2: exponentials and P, one 32-key chunk at a time ----
+    const float ref = (m == -CUDART_INF_F) ? 0.f : m;
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    const float2 nr2 = make_float2(-ref, -ref);
+    float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int cc = 0; cc < PP_BN / 32; ++cc) {
+        uint32_t pk[16];
+        if (live(cc)) {
+            float sr[32];
+            tmem_ld32(s_addr + cc * 32, sr);
+            tmem_ld_wait_dep(sr);
+            mask32(sr, cc);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                float2 y = fma2(make_float2(sr[e], sr[e + 1]), sc2, nr2);
+                if ((e / 2) % PP_POLY_EVERY == PP_POLY_EVERY - 1) {
+                    y = exp2_poly2(y);
+                } else {
+                    y.x = ex2_approx(y.x);
+                    y.y = ex2_approx(y.y);
+                }
+                if (e & 2) acc2b = add2(acc2b, y);
+                else acc2 = add2(acc2, y);
+                pk[e / 2] = pack_bf16x2(y.x, y.y);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        }
+        tmem_st16u(s_addr + cc * 16, pk);
+    }
+    const float2 tot = add2(acc2, acc2b);
+    l += tot.x + tot.y;
+}
+
+template <int D>
+__global__ void __maxnreg__(200)
+    swa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                          const TcPrefillArgs a)
+{
+    using C = PCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem + C::OFF_Q;   // Q_X at sQ + X * QTILE
+    uint8_t *sK = smem + C::OFF_K;
+    uint8_t *sV = smem + C::OFF_V;
+    PPBars *bars = reinterpret_cast<PPBars *>(smem + C::OFF_BAR);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const PPWork w = pp_make_work(a);
+    WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < PP_NSTAGE; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_full[x], PP_BM / 32);
+            mbar_init(&bars->pv_done[x], 1);
+            mbar_init(&bars->epi[x], PP_BM / 32);
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&tmO);
+    }
+    if (warp == 9) tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 8) {
+        // ------------------------------------------------------ producer --
+        int kiss[PP_NSTAGE] = {}, viss[PP_NSTAGE] = {};
+        bool ok = true;
+        if (lane == 0) {
+            int nq = 0;
+            for (int x = 0; x < 2; ++x) nq += w.q[x].active ? 1 : 0;
+            mbar_expect_tx(&bars->q_full, nq * C::QTILE);
+            for (int x = 0; x < 2; ++x)
+                if (w.q[x].active)
+                    for (int ch = 0; ch < C::NCH; ++ch) {
+                        SWA_DCHECK(w.q[x].m0 >= 0 && w.q[x].m0 < a.T && w.q[x].h < a.Hq, a.ctl.status);
+                        tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, &tmQ, &bars->q_full, ch * C::E, w.q[x].h,
+                                    w.q[x].m0, w.b);
+                    }
+        }
+        for (int t = 0; t < w.n_tiles && ok; ++t) {
+            const int key0 = (w.j_lo + t) * PP_BN;
+            const int st = t % PP_NSTAGE;
+            const uint32_t par = ((t / PP_NSTAGE) & 1) ^ 1;
+            ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
+            if (!ok) break;
+            SWA_DCHECK(key0 >= 0 && key0 < a.T, a.ctl.status);
+            if (lane == 0) {
+                mbar_expect_tx(&bars->k_full[st], C::KTILE);
+                for (int ch = 0; ch < C::NCH; ++ch)
+                    tma_load_4d(sK + st * C::KTILE + ch * C::KCH, &tmK, &bars->k_full[st], ch * C::E, w.hk, key0, w.b);
+            }
+            kiss[st]++;
+            ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_expect_tx(&bars->v_full[st], C::KTILE);
+                for (int ch = 0; ch < C::NCH; ++ch)
+                    tma_load_4d(sV + st * C::KTILE + ch * C::KCH, &tmV, &bars->v_full[st], ch * C::E, w.hk, key0, w.b);
+            }
+            viss[st]++;
+        }
+        if (!ok && lane == 0) {
+            // let our own copies land before the CTA's shared memory goes away
+            for (int s = 0; s < PP_NSTAGE; ++s) {
+                if (kiss[s] > 0) pp_drain_wait(&bars->k_full[s], (kiss[s] - 1) & 1, a.ctl.limit_ns);
+                if (viss[s] > 0) pp_drain_wait(&bars->v_full[s], (viss[s] - 1) & 1, a.ctl.limit_ns);
+            }
+        }
+    } else if (warp == 9) {
+        // ----------------------------------------------------------- MMA --
+        // The whole warp runs the schedule (waits, descriptor arithmetic) in
+        // lock step; lane 0 alone issues MMAs and commits.
+        constexpr uint32_t idesc_qk = umma_idesc_bf16(PP_BM, PP_BN, 0, 0);
+        constexpr uint32_t idesc_pv = umma_idesc_bf16(PP_BM, D, 0, 1);
+        // descriptors are built once; a k-step or stage only adds a constant
+        // to the 14-bit start-address field (addresses < 2^18)
+        const uint64_t dq0 = umma_smem_desc(smem_u32(sQ), 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dk0 = umma_smem_desc(smem_u32(sK), 16, 8 * C::RB, C::LAYOUT);
+        const uint64_t dv0 = umma_smem_desc(smem_u32(sV), C::KCH, 8 * C::RB, C::LAYOUT);
+        const bool leader = lane == 0;
+        int cnt[2] = {0, 0};   // key tiles each query tile has multiplied by V so far
+        bool ok = warp_wait_bounded(&bars->q_full, 0, ctl);
+        auto qk = [&](int x, int t) {
+            const int st = t % PP_NSTAGE;
+            const uint64_t dq = dq0 + (uint64_t)((x * C::QTILE) >> 4);
+            const uint64_t dk = dk0 + (uint64_t)((st * C::KTILE) >> 4);
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int byte = kk * 32;
+                    const uint64_t qo = (uint64_t)(((byte / C::RB) * C::QCH + (byte % C::RB)) >> 4);
+                    const uint64_t ko = (uint64_t)(((byte / C::RB) * C::KCH + (byte % C::RB)) >> 4);
+                    mma_bf16_ss(tmem + pp_col_s(x), dq + qo, dk + ko, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars->s_full[x]);
+            }
+        };
+        auto pv = [&](int x, int t) -> bool {
+            if (!warp_wait_bounded(&bars->p_full[x], cnt[x] & 1, ctl)) return false;
+            tc_fence_after();
+            const int st = t % PP_NSTAGE;
+            const uint64_t dv = dv0 + (uint64_t)((st * C::KTILE) >> 4);
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < PP_BN / 16; ++kk)
+                    mma_bf16_ts(tmem + pp_col_o(x), tmem + pp_col_s(x) + kk * 8,
+                                dv + (uint64_t)((kk * 16 * C::RB) >> 4), idesc_pv, (cnt[x] > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars->pv_done[x]);
+            }
+            cnt[x]++;
+            return true;
+        };
+        // prologue: QK^T of the first key tile for both query tiles
+        if (ok && w.n_tiles > 0) {
+            ok = warp_wait_bounded(&bars->k_full[0], 0, ctl);
+            if (ok) {
+                tc_fence_after();
+                for (int x = 0; x < 2; ++x)
+                    if (pp_active(w.q[x], 0)) qk(x, 0);
+                if (leader) mma_commit(&bars->k_empty[0]);
+            }
+        }
+        for (int t = 0; t < w.n_tiles && ok; ++t) {
+            const int st = t % PP_NSTAGE;
+            const bool more = t + 1 < w.n_tiles;
+            ok = warp_wait_bounded(&bars->v_full[st], (t / PP_NSTAGE) & 1, ctl);
+            if (!ok) break;
+            // tile A: PV of key tile t, then QK^T of key tile t+1 into the
+            // same S columns (issue order keeps them apart)
+            if (pp_active(w.q[0], t)) ok = pv(0, t);
+            if (!ok) break;
+            if (more) {
+                ok = warp_wait_bounded(&bars->k_full[(t + 1) % PP_NSTAGE], ((t + 1) / PP_NSTAGE) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                if (pp_active(w.q[0], t + 1)) qk(0, t + 1);
+            }
+            // tile B likewise, half a step behind
+            if (pp_active(w.q[1], t)) ok = pv(1, t);
+            if (!ok) break;
+            if (leader) mma_commit(&bars->v_empty[st]);
+            if (more) {
+                if (pp_active(w.q[1], t + 1)) qk(1, t + 1);
+                if (leader) mma_commit(&bars->k_empty[(t + 1) % PP_NSTAGE]);
+            }
+            __syncwarp();
+        }
+        // all MMAs lane 0 issued are complete before TMEM is freed
+        if (leader) {
+            mma_commit(&bars->drain);
+            pp_drain_wait(&bars->drain, 0, a.ctl.limit_ns);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------- softmax + epilogue --
+        const int x = warp / 4;                 // query tile of this warpgroup
+        const int quarter = warp % 4;
+        const int r = quarter * 32 + lane;      // row in tile = TMEM lane
+        const PPTile qt = w.q[x];
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + pp_col_s(x);
+        const uint32_t o_addr = tmem + lane_off + pp_col_o(x);
+        const int i_row = qt.m0 + r;            // query position
+        const bool row_real = qt.active && r < qt.nrows;
+        const bool warp_has_rows = qt.active && quarter * 32 < qt.nrows;
+        const int wi0 = qt.m0 + quarter * 32, wi1 = wi0 + 31;
+        float m = -CUDART_INF_F, l = 0.f;
+        bool ok = true;
+        int c = 0;
+        for (int t = 0; t < w.n_tiles && qt.active; ++t) {
+            if (!pp_active(qt, t)) continue;
+            ok = warp_wait_bounded(&bars->s_full[x], c & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            // which 32-key chunks can any row of this warp see
+            const int key0 = (w.j_lo + t) * PP_BN;
+            int c_lo = 0, c_hi = -1;
+            bool interior = false;
+            if (warp_has_rows) {
+                const int lo = max(max(key0, wi0 - a.left), 0);
+                const int hi = min(min(key0 + PP_BN - 1, wi1 + a.right), a.T - 1);
+                if (lo <= hi) {
+                    c_lo = (lo - key0) / 32;
+                    c_hi = (hi - key0) / 32;
+                }
+                interior = (key0 + PP_BN - 1 < a.T) && band_contains(wi1, key0, a.left, a.right) &&
+                           band_contains(wi0, key0 + PP_BN - 1, a.left, a.right);
+            }
+            SWA_DCHECK(c_lo >= 0 && c_hi < PP_BN / 32, a.ctl.status);
+            // visible columns of this row
+            const int col_lo = max(i_row - a.left - key0, 0);
+            const int col_hi = min(min(i_row + a.right, a.T - 1) - key0, PP_BN - 1);
+            bool rescale_o;
+            float alpha;
+            if (interior && c_lo == 0 && c_hi == PP_BN / 32 - 1)
+                pp_softmax_tile<true>(s_addr, c_lo, c_hi, col_lo, col_hi, a.scale_log2, m, l, rescale_o, alpha,
+                                      c == 0);
+            else
+                pp_softmax_tile<false>(s_addr, c_lo, c_hi, col_lo, col_hi, a.scale_log2, m, l, rescale_o, alpha,
+                                       c == 0);
+            // O rescale (rare): wait for the previous tile's PV, which
+            // accumulates into O; this tile's PV waits for P
+            if (__any_sync(0xffffffffu, rescale_o)) {
+                ok = warp_wait_bounded(&bars->pv_done[x], (c - 1) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                const float f = rescale_o ? alpha : 1.f;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 16; ++cc) {
+                    float ov[16];
+                    tmem_ld16(o_addr + cc * 16, ov);
+                    tmem_ld_wait_dep16(ov);
+                    uint32_t ou[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(ov[e] * f);
+                    tmem_st16u(o_addr + cc * 16, ou);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full[x]);
+            c++;
+        }
+
+        // ---- epilogue: O / l -> bf16 -> shared memory -> TMA store ----
+        if (ok && c > 0) ok = warp_wait_bounded(&bars->pv_done[x], (c - 1) & 1, ctl);
+        uint8_t *stage = sQ + x * C::QTILE;    // Q_X is no longer read: its last QK^T is complete
+        if (ok && qt.active) {
+            tc_fence_after();
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 16; ++cc) {
+                float ov[16];
+                tmem_ld16(o_addr + cc * 16, ov);
+                tmem_ld_wait_dep16(ov);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(ov[u * 8 + 0] * inv, ov[u * 8 + 1] * inv);
+                    pk.y = pack_bf16x2(ov[u * 8 + 2] * inv, ov[u * 8 + 3] * inv);
+                    pk.z = pack_bf16x2(ov[u * 8 + 4] * inv, ov[u * 8 + 5] * inv);
+                    pk.w = pack_bf16x2(ov[u * 8 + 6] * inv, ov[u * 8 + 7] * inv);
+                    *reinterpret_cast<uint4 *>(stage + pp_tile_offset<D>(r, cc * 16 + u * 8, C::QCH)) = pk;
+                }
+            }
+            if (a.lse && row_real)
+                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_row] =
+                    (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
+        }
+        // staging tile complete -> one thread per warpgroup stores it
+        // (rows past T are clipped by the tensor map; an abort anywhere in
+        // the CTA skips the store)
+        if (qt.active) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->epi[x]);
+            if (r == 0 && wait_bounded(&bars->epi[x], 0, ctl) && !bars->abort) {
+                for (int ch = 0; ch < C::NCH; ++ch)
+                    tma_store_4d(&tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
+                tma_store_commit();
+                tma_store_wait_all();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int D>
+cudaError_t launch_pp_d(const TcPrefillArgs &a, cudaStream_t s)
+{
+    using C = PCfg<D>;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq, D, PP_BM) || !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv, D, PP_BN) ||
+        !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv, D, PP_BN) || !make_bthd_map(&mo, a.o, a.B, a.T, a.Hq, D, PP_BM))
+        return cudaErrorInvalidValue;
+    static DeviceOnce once;
+    cudaError_t e = once.get(
+        [&](int) {
+            return cudaFuncSetAttribute(swa_prefill_pp_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::SMEM_BYTES);
+        },
+        nullptr);
+    if (e != cudaSuccess) return e;
+    const int G = a.Hq / a.Hkv;
+    const int nqt = (a.T + PP_BM - 1) / PP_BM;
+    const long long units = (long long)a.B * ((G % 2 == 0) ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
+    if (units == 0) return cudaSuccess;
+    if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    swa_prefill_pp_kernel<D><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_pp_applies(int d, const TcPrefillArgs &a)
+{
+    return (d == 64 || d == 128) && a.gidx == nullptr && a.g == 0;
+}
+
+cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s)
+{
+    switch (d) {
+    case 64: return launch_pp_d<64>(a, s);
+    case 128: return launch_pp_d<128>(a, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace swa

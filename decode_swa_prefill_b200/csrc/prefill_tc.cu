@@ -172,6 +172,22 @@ __device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
     return q.active ? (q.te - q.ts) + n_glob : 0;
 }
 
+// Is packed sequence b's entry consistent (offsets inside the rows and
+// non-decreasing, length at most max_len, window at least 1)?
+__device__ __forceinline__ bool varlen_ok(const VarlenArgs &vl, int b, int total)
+{
+    const int c0 = vl.cu[b], c1 = vl.cu[b + 1];
+    return c0 >= 0 && c1 >= c0 && c1 <= total && c1 - c0 <= vl.max_len && (!vl.wseq || vl.wseq[b] >= 1);
+}
+
+// Keys before the query a row of packed sequence b sees: its own window's
+// (clipped to the longest sequence, like the call's single window), or the
+// call's.
+__device__ __forceinline__ int varlen_left(const VarlenArgs &vl, int b, int left)
+{
+    return vl.wseq ? min(max(vl.wseq[b], 1) - 1, vl.max_len) : left;
+}
+
 template <bool RING, bool SINKS, bool VARLEN>
 __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl,
                                           int n_mode1)
@@ -255,11 +271,13 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs
         } else {
             // sequence length (a packed sequence: its own; tiles past it idle)
             int TT = a.T;
+            int left = a.left;
             if constexpr (VARLEN) {
                 // an inconsistent entry (decreasing, past the rows, longer
-                // than max_len) makes the sequence empty; the CTA reports it
-                const int c0 = vl.cu[w.b], c1 = vl.cu[w.b + 1];
-                TT = (c0 < 0 || c1 < c0 || c1 > a.T || c1 - c0 > vl.max_len) ? 0 : c1 - c0;
+                // than max_len, a window below 1) makes the sequence empty;
+                // the CTA reports it
+                TT = varlen_ok(vl, w.b, a.T) ? vl.cu[w.b + 1] - vl.cu[w.b] : 0;
+                left = varlen_left(vl, w.b, a.left);
                 for (int x = 0; x < 2; ++x) {
                     if (w.q[x].m0 >= TT) w.q[x].active = false;
                     w.q[x].nrows = min(BM, TT - w.q[x].m0);
@@ -271,7 +289,7 @@ __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs
             int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
             for (int x = 0; x < 2; ++x) {
                 if (!w.q[x].active) continue;
-                lo_x[x] = max(0, w.q[x].m0 - a.left);
+                lo_x[x] = max(0, w.q[x].m0 - left);
                 hi_x[x] = min(TT - 1, w.q[x].m0 + BM - 1 + a.right);
                 lo = min(lo, lo_x[x]);
                 hi = max(hi, hi_x[x]);
@@ -307,12 +325,14 @@ __device__ __forceinline__ int tile_cols(const Work &w, const TcPrefillArgs &a, 
 template <int D>
 __device__ __forceinline__ void gather_tile(uint8_t *dst, int rows, int ch_bytes, const __nv_bfloat16 *base,
                                             const int32_t *rows_idx, int nrows, int b, int T, int H, int head,
-                                            int lane)
+                                            int lane, int *status)
 {
     constexpr int GR = D / 8; // 16-byte granules per row
+    (void)status;
     for (int idx = lane; idx < rows * GR; idx += 32) {
         const int r = idx / GR, u = idx % GR;
         const long long pos = r < nrows ? rows_idx[r] : 0;
+        SWA_DCHECK(pos >= 0 && pos < T, status);
         const __nv_bfloat16 *src = base + (((long long)b * T + pos) * H + head) * D + u * 8;
         cp_async16(dst + tile_offset<D>(r, u * 8, ch_bytes), src, r < nrows ? 16u : 0u);
     }
@@ -471,10 +491,10 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
     const int lane = threadIdx.x % 32;
     const Work w = make_work<RING, SINKS, VARLEN>(a, ring, vl, n_mode1);
     if constexpr (VARLEN) {
-        const int c0 = vl.cu[w.b], c1 = vl.cu[w.b + 1];
-        if ((c0 < 0 || c1 < c0 || c1 > a.T || c1 - c0 > vl.max_len) && threadIdx.x == 0)
-            atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+        if (!varlen_ok(vl, w.b, a.T) && threadIdx.x == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     }
+    // keys before the query (packed sequences: the sequence's own window)
+    const int left = VARLEN ? varlen_left(vl, w.b, a.left) : a.left;
     // a packed-sequence unit past its sequence's end has nothing to do
     if (VARLEN && !w.q[0].active) return;
     const int tb = VARLEN ? 0 : w.b;         // batch coordinate of the tensors
@@ -526,16 +546,18 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                 for (int x = 0; x < 2; ++x) nq += w.q[x].active ? 1 : 0;
                 mbar_expect_tx(&bars->q_full, nq * C::QTILE);
                 for (int x = 0; x < 2; ++x)
-                    if (w.q[x].active)
+                    if (w.q[x].active) {
+                        SWA_DCHECK(w.q[x].m0 >= 0 && w.q[x].m0 < a.T && w.q[x].h < a.Hq, a.ctl.status);
                         for (int ch = 0; ch < C::NCH; ++ch)
                             tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, tmQ, &bars->q_full, ch * C::E, w.q[x].h,
                                         w.q[x].m0 + trow0, tb);
+                    }
             }
         } else {
             for (int x = 0; x < 2; ++x)
                 if (w.q[x].active)
                     gather_tile<D>(sQ + x * C::QTILE, BM, C::QCH, static_cast<const __nv_bfloat16 *>(a.q),
-                                   gb + w.q[x].gt * BM, w.q[x].nrows, w.b, a.T, a.Hq, w.q[x].h, lane);
+                                   gb + w.q[x].gt * BM, w.q[x].nrows, w.b, a.T, a.Hq, w.q[x].h, lane, a.ctl.status);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->q_full);
@@ -553,12 +575,15 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                 if (t >= w.n_band) {
                     const int gt = t - w.n_band;
                     gather_tile<D>(dst, BN, C::KCH, src, gb + gt * BN, min(BN, a.g - gt * BN), w.b, a.T, a.Hkv, w.hk,
-                                   lane);
+                                   lane, a.ctl.status);
                 } else {
                     const long long key0 = (long long)(w.j_lo + t) * BN;
                     const bool ring_tile = RING && key0 < w.p0;
                     const long long slot0 = ring_tile ? key0 % ring.W : 0;
                     if (!RING || !ring_tile || (key0 + BN <= w.p0 && slot0 + BN <= ring.W)) {
+                        SWA_DCHECK(ring_tile ? (slot0 >= 0 && slot0 + BN <= ring.W)
+                                             : (key0 >= p0 && key0 - p0 < a.T),
+                                   a.ctl.status);
                         if (lane == 0) {
                             mbar_expect_tx(bar, C::KTILE);
                             for (int ch = 0; ch < C::NCH; ++ch) {
@@ -610,6 +635,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                 ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
                 if (!ok) break;
                 if (band) {
+                    SWA_DCHECK(key0 >= 0 && key0 < w.kend, a.ctl.status);
                     if (lane == 0) {
                         mbar_expect_tx(&bars->k_full[st], C::KTILE);
                         for (int ch = 0; ch < C::NCH; ++ch)
@@ -622,7 +648,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                                         a.T, a.Hkv, w.hk, lane);
                     else
                         gather_tile<D>(sK + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.k),
-                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane, a.ctl.status);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->k_full[st]);
@@ -643,7 +669,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                                         a.T, a.Hkv, w.hk, lane);
                     else
                         gather_tile<D>(sV + st * C::KTILE, BN, C::KCH, static_cast<const __nv_bfloat16 *>(a.v),
-                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane);
+                                       gb + gt * BN, nr, w.b, a.T, a.Hkv, w.hk, lane, a.ctl.status);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->v_full[st]);
@@ -781,18 +807,19 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                     c_hi = (int)((min(key0 + BN - 1, KEND - 1) - key0) / 32);
                     interior = key0 + BN <= KEND;
                 } else if (band) {
-                    const long long lo = max(max((long long)key0, wi0 - a.left), 0LL);
+                    const long long lo = max(max((long long)key0, wi0 - left), 0LL);
                     const long long hi = min(min((long long)key0 + BN - 1, wi1 + a.right), (long long)KEND - 1);
                     if (lo <= hi) {
                         c_lo = (int)((lo - key0) / 32);
                         c_hi = (int)((hi - key0) / 32);
                     }
-                    interior = (key0 + BN - 1 < KEND) && band_contains(wi1, key0, a.left, a.right) &&
-                               band_contains(wi0, key0 + BN - 1, a.left, a.right);
+                    interior = (key0 + BN - 1 < KEND) && band_contains(wi1, key0, left, a.right) &&
+                               band_contains(wi0, key0 + BN - 1, left, a.right);
                 } else {
                     c_hi = (min(BN, a.g - (t - w.n_band) * BN) - 1) / 32;
                 }
             }
+            SWA_DCHECK(c_lo >= 0 && c_hi < BN / 32, a.ctl.status);
             // visible columns of this row as one int range (band, dense)
             TileCtx k;
             k.s_addr = tmem + lane_off + col_s(x, b);
@@ -804,7 +831,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
             if (w.mode == 1) {
                 k.col_hi = (int)min((kpos_t)BN - 1, KEND - 1 - key0);
             } else if (band) {
-                k.col_lo = (int)max(i_row - a.left - key0, 0LL);
+                k.col_lo = (int)max(i_row - left - key0, 0LL);
                 k.col_hi = (int)min(min(i_row + a.right, (long long)KEND - 1) - key0, (long long)BN - 1);
             }
             k.gc_base = (t - w.n_band) * BN;
@@ -882,6 +909,7 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
                     const int e = cc * 16 + u * 8;
                     if (direct) {
                         if (!skip_row) {
+                            SWA_DCHECK(trow0 + i_out >= 0 && trow0 + i_out < a.T, a.ctl.status);
                             __nv_bfloat16 *dst = o + (((long long)tb * a.T + trow0 + i_out) * a.Hq + qt.h) * D + e;
                             *reinterpret_cast<uint4 *>(dst) = pk;
                         }
@@ -1098,6 +1126,7 @@ cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const Rin
 {
     // a causal window of at most 64 keys: the single-pass kernel
     if (mode == 0 && ring.pos == nullptr && prefill_narrow_applies(d, a)) return launch_prefill_narrow(d, a, s);
+
     switch (d) {
     case 32: return launch_d<32>(mode, a, ring, s);
     case 64: return launch_d<64>(mode, a, ring, s);

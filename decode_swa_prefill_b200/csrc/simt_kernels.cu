@@ -41,7 +41,9 @@ __global__ void mask_export_kernel(uint8_t *mask, int T, int left, int right, co
 // --------------------------------------------------------- cache append --
 // Token t of row b goes to slot (pos[b]+t) mod W (Ultralytics ring-buffer
 // paragraph); with n > W only the last W tokens are copied, so no two
-// threads write one slot.  16-byte units.
+// threads write one slot.  16-byte units.  A paged ring keeps slot s of
+// sequence b in row s mod P of page ptable[b][s/P] of the pool; a page outside
+// the pool is reported in the status word and its token is not written.
 __global__ void append_kernel(AppendArgs a)
 {
     const int upr = a.row_bytes / 16;
@@ -70,8 +72,20 @@ __global__ void append_kernel(AppendArgs a)
             continue;
         }
         const long long slot = (p + t) % a.W;
+        SWA_DCHECK(slot >= 0 && slot < a.W && t >= 0 && t < a.n, a.ctl.status);
+        long long row;  // destination row of the cache or pool
+        if (a.ptable) {
+            const int pg = a.ptable[(long long)b * (a.W >> a.page_shift) + (slot >> a.page_shift)];
+            if ((unsigned)pg >= (unsigned)a.num_pages) {
+                if (u == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+                continue;
+            }
+            row = (((long long)pg * a.Hkv + hk) << a.page_shift) + (slot & ((1LL << a.page_shift) - 1));
+        } else {
+            row = ((long long)b * a.Hkv + hk) * a.W + slot;
+        }
         const long long src = (((long long)b * a.n + t) * a.Hkv + hk) * a.row_bytes + u * 16;
-        const long long dst = (((long long)b * a.Hkv + hk) * a.W + slot) * a.row_bytes + u * 16;
+        const long long dst = row * a.row_bytes + u * 16;
         const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.kn) + src));
         const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(a.vn) + src));
         *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(a.kc) + dst) = kv;
@@ -150,6 +164,7 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
     } else {
         const long long ip = p0 + i;  // absolute position of the row
         long long first = 0, last = p0 + a.T - 1;  // the row's sequence
+        int left = a.left;
         if (a.cu) {
             // packed sequences: the one holding row i (kept inside the rows
             // even for an inconsistent cu)
@@ -161,8 +176,18 @@ __global__ void __launch_bounds__(32 * F32_ROWS_PER_CTA)
             }
             first = max(0LL, (long long)a.cu[s0]);
             last = min((long long)a.T - 1, (long long)a.cu[s0 + 1] - 1);
+            if (a.wseq) {
+                // the sequence's own window; below 1: rows left untouched,
+                // reported in the status word
+                const int wv = a.wseq[s0];
+                if (wv < 1) {
+                    if (lane == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+                    return;
+                }
+                left = (int)min((long long)wv - 1, (long long)a.left);
+            }
         }
-        const long long lo = max(first, ip - a.left);
+        const long long lo = max(first, ip - left);
         const long long hi = min(last, ip + a.right);
         if (!gb && a.g > 0)  // sinks older than the window
             for (long long j = 0; j < min((long long)a.g, lo); ++j) visit(j);
@@ -226,10 +251,107 @@ struct Ld<float> {
     __device__ __forceinline__ static void store(float *p, float x) { *p = x; }
 };
 
-template <typename T, int D, int G, bool SINKS>
+// Where a decode reads its key/value rows: the dense ring, the dense ring
+// plus sink caches, or a paged ring (pool + page table).
+constexpr int SRC_RING = 0, SRC_SINKS = 1, SRC_PAGED = 2;
+
+// Row (in rows of d elements) of ring slot sl of (sequence b, kv head hk) in
+// a paged pool; a page outside the pool reads page 0 and sets *bad.
+__device__ __forceinline__ long long paged_row(const DecodeArgs &a, const int32_t *tbl, int hk, int sl, bool *bad)
+{
+    int pg = __ldg(tbl + (sl >> a.page_shift));
+    if ((unsigned)pg >= (unsigned)a.num_pages) {
+        *bad = true;
+        pg = 0;
+    }
+    return (((long long)pg * a.Hkv + hk) << a.page_shift) + (sl & ((1 << a.page_shift) - 1));
+}
+
+// The end of a decode CTA: merge the warps' partials (running max m in log2
+// units, sum l, unnormalised accumulator) held in shared memory, then
+//  - one split: write o (and lse);
+//  - splits in one thread-block cluster (a.cluster): keep the CTA's merged
+//    partial in shared memory; after a cluster barrier each CTA of the
+//    cluster merges a 1/splits slice of the G*D outputs, reading every
+//    split's partial from its CTA's shared memory (distributed shared
+//    memory), and writes o; a second barrier keeps every CTA's shared memory
+//    alive until the others have read it.  No workspace, no second launch.
+//  - otherwise: write the split's partial to the workspace for
+//    decode_combine_kernel.
+// The LSE merge: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+template <typename T, int D, int G>
+__device__ __forceinline__ void decode_finish(const DecodeArgs &a, int b, int hk, int split,
+                                              const float (*sm_m)[G], const float (*sm_l)[G],
+                                              const float (*sm_acc)[G][D])
+{
+    __shared__ float cm[G], cl[G], co[G][D];   // this CTA's merged partial (cluster merge)
+    const int Hq = a.Hq;
+    const bool cluster = a.cluster && a.splits > 1;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, e = idx % D;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, sm_m[w][g]);
+        const float Mu = M == -CUDART_INF_F ? 0.f : M;
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) {
+            const float f = ex2_approx(sm_m[w][g] - Mu);
+            L += sm_l[w][g] * f;
+            O += sm_acc[w][g][e] * f;
+        }
+        const int h = hk * G + g;
+        if (a.splits == 1) {
+            T *o = static_cast<T *>(a.o) + ((long long)b * Hq + h) * D;
+            Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
+            if (a.lse && e == 0)
+                a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+        } else if (cluster) {
+            co[g][e] = O;
+            if (e == 0) {
+                cm[g] = M;
+                cl[g] = L;
+            }
+        } else {
+            float *part = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
+            part[e] = O;
+            if (e == 0) {
+                part[D] = M;
+                part[D + 1] = L;
+            }
+        }
+    }
+    if (!cluster) return;
+    cluster_sync();
+    const int S = a.splits;
+    const int per = G * D / S;               // outputs this CTA merges
+    const int r0 = (int)cluster_ctarank() * per;
+    for (int idx = r0 + threadIdx.x; idx < r0 + per; idx += blockDim.x) {
+        const int g = idx / D, e = idx % D;
+        float M = -CUDART_INF_F;
+        for (int q = 0; q < S; ++q) M = fmaxf(M, ld_cluster_f32(cluster_peer_addr(&cm[g], q)));
+        const float Mu = M == -CUDART_INF_F ? 0.f : M;
+        float L = 0.f, O = 0.f;
+        for (int q = 0; q < S; ++q) {
+            const float f = ex2_approx(ld_cluster_f32(cluster_peer_addr(&cm[g], q)) - Mu);
+            L += ld_cluster_f32(cluster_peer_addr(&cl[g], q)) * f;
+            O += ld_cluster_f32(cluster_peer_addr(&co[g][e], q)) * f;
+        }
+        const int h = hk * G + g;
+        T *o = static_cast<T *>(a.o) + ((long long)b * Hq + h) * D;
+        Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
+        if (a.lse && e == 0)
+            a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
+    }
+    cluster_sync();
+}
+
+template <typename T, int D, int G, int SRC>
 __global__ void __launch_bounds__(32 * DEC_WARPS)
     decode_kernel(DecodeArgs a)
 {
+    constexpr bool SINKS = SRC == SRC_SINKS;
+    constexpr bool PAGED = SRC == SRC_PAGED;
     constexpr int EPL = D / 32;
     constexpr int NB = 32 / G;
     const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -251,12 +373,16 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const T *kb = static_cast<const T *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const T *vb = static_cast<const T *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
+    const int32_t *tbl = PAGED ? a.ptable + (long long)b * (a.W >> a.page_shift) : nullptr;
+    bool bad_page = false;
     auto krow = [&](int sl) -> const T * {
         if (SINKS && sl >= n_valid) return static_cast<const T *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
+        if (PAGED) return static_cast<const T *>(a.kc) + paged_row(a, tbl, hk, sl, &bad_page) * D;
         return kb + (long long)sl * D;
     };
     auto vrow = [&](int sl) -> const T * {
         if (SINKS && sl >= n_valid) return static_cast<const T *>(a.vs) + sink0 + (long long)(sl - n_valid) * D;
+        if (PAGED) return static_cast<const T *>(a.vc) + paged_row(a, tbl, hk, sl, &bad_page) * D;
         return vb + (long long)sl * D;
     };
 
@@ -282,6 +408,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
 #pragma unroll
         for (int n = 0; n < NB; ++n) {
             const int sl = min(base + n, s_end - 1); // clamp: masked below
+            SWA_DCHECK(sl >= 0 && sl < (SINKS ? a.W + a.n_sink : a.W), a.ctl.status);
             Ld<T>::template row<EPL>(krow(sl) + lane * EPL, kr[n]);
             Ld<T>::template row<EPL>(vrow(sl) + lane * EPL, vr[n]);
         }
@@ -346,6 +473,8 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
             }
     }
 
+    if (PAGED && bad_page) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+
     // merge the warps' partials in shared memory
     __shared__ float sm_m[DEC_WARPS][G], sm_l[DEC_WARPS][G];
     __shared__ float sm_acc[DEC_WARPS][G][D];
@@ -360,34 +489,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
 #pragma unroll
         for (int e = 0; e < EPL; ++e) sm_acc[warp][g][lane * EPL + e] = acc[g][e];
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int g = idx / D, e = idx % D;
-        float M = -CUDART_INF_F;
-#pragma unroll
-        for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, sm_m[w][g]);
-        const float Mu = M == -CUDART_INF_F ? 0.f : M;
-        float L = 0.f, O = 0.f;
-#pragma unroll
-        for (int w = 0; w < DEC_WARPS; ++w) {
-            const float f = ex2_approx(sm_m[w][g] - Mu);
-            L += sm_l[w][g] * f;
-            O += sm_acc[w][g][e] * f;
-        }
-        const int h = hk * G + g;
-        if (a.splits == 1) {
-            T *o = static_cast<T *>(a.o) + ((long long)b * Hq + h) * D;
-            Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
-            if (a.lse && e == 0)
-                a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
-        } else {
-            float *part = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
-            part[e] = O;
-            if (e == 0) {
-                part[D] = M;
-                part[D + 1] = L;
-            }
-        }
-    }
+    decode_finish<T, D, G>(a, b, hk, split, sm_m, sm_l, sm_acc);
 }
 
 // bf16 decode with 16-byte loads (used when G <= d/8).  A row of d bf16 is
@@ -416,10 +518,12 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w)
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-template <int D, int G, bool SINKS>
+template <int D, int G, int SRC>
 __global__ void __launch_bounds__(32 * DEC_WARPS)
     decode_bf16_kernel(DecodeArgs a)
 {
+    constexpr bool SINKS = SRC == SRC_SINKS;
+    constexpr bool PAGED = SRC == SRC_PAGED;
     constexpr int LPR = D / 8;          // lanes per row
     constexpr int RPW = 32 / LPR;       // rows per warp load
     constexpr int NBL = LPR / G;        // slots per lane per batch
@@ -446,10 +550,18 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.kc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.vc) + ((long long)b * a.Hkv + hk) * (long long)a.W * D;
     const long long sink0 = ((long long)b * a.Hkv + hk) * (long long)a.n_sink * D;
-    // row sources: the ring, or (the last split of a call with sinks) the
-    // ring and then the sink caches
-    auto ring_k = [&](int sl) -> const __nv_bfloat16 * { return kb + (long long)sl * D; };
-    auto ring_v = [&](int sl) -> const __nv_bfloat16 * { return vb + (long long)sl * D; };
+    // row sources: the ring (dense, or paged through the page table), or
+    // (the last split of a call with sinks) the ring and then the sink caches
+    const int32_t *tbl = PAGED ? a.ptable + (long long)b * (a.W >> a.page_shift) : nullptr;
+    bool bad_page = false;
+    auto ring_k = [&](int sl) -> const __nv_bfloat16 * {
+        if (PAGED) return static_cast<const __nv_bfloat16 *>(a.kc) + paged_row(a, tbl, hk, sl, &bad_page) * D;
+        return kb + (long long)sl * D;
+    };
+    auto ring_v = [&](int sl) -> const __nv_bfloat16 * {
+        if (PAGED) return static_cast<const __nv_bfloat16 *>(a.vc) + paged_row(a, tbl, hk, sl, &bad_page) * D;
+        return vb + (long long)sl * D;
+    };
     auto tail_k = [&](int sl) -> const __nv_bfloat16 * {
         if (sl >= n_valid) return static_cast<const __nv_bfloat16 *>(a.ks) + sink0 + (long long)(sl - n_valid) * D;
         return kb + (long long)sl * D;
@@ -478,6 +590,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
 #pragma unroll
         for (int n = 0; n < NBL; ++n) {
             const int sl = min(base + n * RPW + rgrp, s_end - 1); // clamp: masked below
+            SWA_DCHECK(sl >= 0 && sl < (SINKS ? a.W + a.n_sink : a.W), a.ctl.status);
             kr[n] = __ldg(reinterpret_cast<const uint4 *>(krow(sl) + part * 8));
             vr[n] = __ldg(reinterpret_cast<const uint4 *>(vrow(sl) + part * 8));
         }
@@ -556,6 +669,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     } else {
         run(ring_k, ring_v);
     }
+    if (PAGED && bad_page) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
     // sum the row groups' accumulators (same softmax reference per head)
 #pragma unroll
     for (int k = LPR; k < 32; k <<= 1)
@@ -585,34 +699,7 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
                 sm_acc[warp][g][part * 8 + 2 * e + 1] = acc[g][e].y;
             }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-        const int g = idx / D, e = idx % D;
-        float M = -CUDART_INF_F;
-#pragma unroll
-        for (int w2 = 0; w2 < DEC_WARPS; ++w2) M = fmaxf(M, sm_m[w2][g]);
-        const float Mu = M == -CUDART_INF_F ? 0.f : M;
-        float L = 0.f, O = 0.f;
-#pragma unroll
-        for (int w2 = 0; w2 < DEC_WARPS; ++w2) {
-            const float f = ex2_approx(sm_m[w2][g] - Mu);
-            L += sm_l[w2][g] * f;
-            O += sm_acc[w2][g][e] * f;
-        }
-        const int h = hk * G + g;
-        if (a.splits == 1) {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(a.o) + ((long long)b * Hq + h) * D;
-            o[e] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-            if (a.lse && e == 0)
-                a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
-        } else {
-            float *part_out = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
-            part_out[e] = O;
-            if (e == 0) {
-                part_out[D] = M;
-                part_out[D + 1] = L;
-            }
-        }
-    }
+    decode_finish<__nv_bfloat16, D, G>(a, b, hk, split, sm_m, sm_l, sm_acc);
 }
 
 // LSE merge of the split partials: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
@@ -636,20 +723,41 @@ __global__ void decode_combine_kernel(DecodeArgs a)
     if (a.lse && e == 0) a.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
 }
 
+// One decode launch: grid (splits, Hkv, B), the splits of a (sequence, kv
+// head) as one cluster along x when they merge in the cluster.
+template <typename K>
+cudaError_t launch_decode_grid(K kernel, const DecodeArgs &a, cudaStream_t s)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.splits, a.Hkv, a.B);
+    cfg.blockDim = dim3(32 * DEC_WARPS, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.cluster ? a.splits : 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
-    dim3 grid(a.splits, a.Hkv, a.B);
-    const bool sinks = a.n_sink > 0;
+    const int src = a.ptable ? SRC_PAGED : a.n_sink > 0 ? SRC_SINKS : SRC_RING;
+    cudaError_t e;
     if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8) {
-        if (sinks) decode_bf16_kernel<D, G, true><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
-        else decode_bf16_kernel<D, G, false><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+        if (src == SRC_PAGED) e = launch_decode_grid(decode_bf16_kernel<D, G, SRC_PAGED>, a, s);
+        else if (src == SRC_SINKS) e = launch_decode_grid(decode_bf16_kernel<D, G, SRC_SINKS>, a, s);
+        else e = launch_decode_grid(decode_bf16_kernel<D, G, SRC_RING>, a, s);
     } else {
-        if (sinks) decode_kernel<T, D, G, true><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
-        else decode_kernel<T, D, G, false><<<grid, 32 * DEC_WARPS, 0, s>>>(a);
+        if (src == SRC_PAGED) e = launch_decode_grid(decode_kernel<T, D, G, SRC_PAGED>, a, s);
+        else if (src == SRC_SINKS) e = launch_decode_grid(decode_kernel<T, D, G, SRC_SINKS>, a, s);
+        else e = launch_decode_grid(decode_kernel<T, D, G, SRC_RING>, a, s);
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || a.splits == 1) return e;
+    if (e != cudaSuccess || a.splits == 1 || a.cluster) return e;
     decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -712,12 +820,14 @@ int decode_splits(int B, int Hq, int Hkv, int d, int W)
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
 {
     const int s = decode_splits(B, Hq, Hkv, d, W);
-    if (s <= 1) return 0;
+    if (s <= kClusterSplits) return 0;   // one split, or merged inside a cluster
     return (size_t)B * Hq * s * (d + 2) * sizeof(float);
 }
 
-cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s)
+cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &args, cudaStream_t s)
 {
+    DecodeArgs a = args;
+    a.cluster = a.splits > 1 && a.splits <= kClusterSplits;
     return dtype_bf16 ? launch_decode_d<__nv_bfloat16>(a, s) : launch_decode_d<float>(a, s);
 }
 

@@ -48,6 +48,16 @@ swa_status from_cuda(cudaError_t e)
 
 size_t elt_size(swa_dtype dt) { return dt == SWA_DTYPE_BF16 ? 2 : 4; }
 
+// log2(page_size) for a paged ring of W slots: page_size a power of two that
+// divides W; -1 otherwise.
+int page_shift_of(int page_size, int W)
+{
+    if (page_size < 1 || (page_size & (page_size - 1)) != 0 || W % page_size != 0) return -1;
+    int sh = 0;
+    while ((1 << sh) < page_size) ++sh;
+    return sh;
+}
+
 bool valid_dtype(swa_dtype dt) { return dt == SWA_DTYPE_BF16 || dt == SWA_DTYPE_F32; }
 
 // Shared checks of the prefill calls.
@@ -121,6 +131,7 @@ const char *swa_status_string(swa_status s)
     case SWA_ERR_UNSUPPORTED: return "unsupported configuration";
     case SWA_ERR_CUDA: return "CUDA error";
     case SWA_ERR_TIMEOUT: return "device wait timed out";
+    case SWA_ERR_INTERNAL: return "device consistency check failed (debug build)";
     }
     return "unknown status";
 }
@@ -243,8 +254,8 @@ swa_status swa_prefill_dilated(const void *q, const void *k, const void *v, void
 }
 
 swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
-                              const int32_t *cu_seqlens, int nseq, int total, int max_seqlen, int Hq, int Hkv, int d,
-                              int W, float scale, swa_dtype dt, void *stream)
+                              const int32_t *cu_seqlens, const int32_t *windows, int nseq, int total, int max_seqlen,
+                              int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream)
 {
     SWA_NVTX_RANGE("swa_prefill_varlen");
     swa_status st = check_prefill(q, k, v, o, lse, 1, total, Hq, Hkv, d, W, scale, dt);
@@ -252,7 +263,11 @@ swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void 
     if (nseq < 0 || max_seqlen < 0 || max_seqlen > total) return SWA_ERR_INVALID_ARG;
     if (nseq == 0 || total == 0 || max_seqlen == 0) return SWA_OK;
     if (!cu_seqlens || !aligned(cu_seqlens, 4)) return SWA_ERR_INVALID_ARG;
-    const int left = W - 1 < max_seqlen ? W - 1 : max_seqlen;
+    if (windows && !aligned(windows, 4)) return SWA_ERR_INVALID_ARG;
+    // with one window per sequence, `left` is the bound every window is
+    // clipped to (a window wider than the longest sequence is the whole
+    // sequence)
+    const int left = windows ? max_seqlen : (W - 1 < max_seqlen ? W - 1 : max_seqlen);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dt == SWA_DTYPE_F32) {
         swa::F32PrefillArgs a{static_cast<const float *>(q), static_cast<const float *>(k),
@@ -260,6 +275,8 @@ swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void 
                               nullptr, 0, scale};
         a.cu = cu_seqlens;
         a.nseq = nseq;
+        a.wseq = windows;
+        if (windows && (st = ctl(&a.ctl)) != SWA_OK) return st;
         return from_cuda(swa::launch_prefill_f32(a, s));
     }
     swa::TcPrefillArgs a{};
@@ -269,7 +286,7 @@ swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void 
     a.lse = lse; a.gidx = nullptr; a.g = 0;
     a.q = q; a.k = k; a.v = v; a.o = o;
     if ((st = ctl(&a.ctl)) != SWA_OK) return st;
-    return from_cuda(swa::launch_prefill_varlen(d, a, swa::VarlenArgs{cu_seqlens, max_seqlen}, s));
+    return from_cuda(swa::launch_prefill_varlen(d, a, swa::VarlenArgs{cu_seqlens, max_seqlen, windows}, s));
 }
 
 swa_status swa_prefill_sinks(const void *q, const void *k, const void *v, void *o, float *lse, int n_sink, int B,
@@ -350,6 +367,28 @@ swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, con
     return from_cuda(swa::launch_append(a, static_cast<cudaStream_t>(stream)));
 }
 
+swa_status swa_cache_append_paged(void *k_pages, void *v_pages, const void *k_new, const void *v_new,
+                                  const int32_t *pos, const int32_t *page_table, int32_t *slot_out, int B, int n,
+                                  int Hkv, int d, int W, int page_size, int num_pages, swa_dtype dt, void *stream)
+{
+    SWA_NVTX_RANGE("swa_cache_append_paged");
+    if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (B < 0 || n < 0 || Hkv < 1 || d < 1 || W < 1 || num_pages < 1) return SWA_ERR_INVALID_ARG;
+    const int shift = page_shift_of(page_size, W);
+    if (shift < 0) return SWA_ERR_INVALID_ARG;
+    if ((d * elt_size(dt)) % 16 != 0) return SWA_ERR_UNSUPPORTED;
+    if (B == 0 || n == 0) return SWA_OK;
+    if (!k_pages || !v_pages || !k_new || !v_new || !pos || !page_table) return SWA_ERR_INVALID_ARG;
+    if (!aligned(k_pages, 16) || !aligned(v_pages, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+        !aligned(pos, 4) || !aligned(page_table, 4) || (slot_out && !aligned(slot_out, 4)))
+        return SWA_ERR_INVALID_ARG;
+    swa::AppendArgs a{k_pages, v_pages, k_new, v_new, pos, slot_out, B, n, Hkv, W,
+                      static_cast<int>(d * elt_size(dt)), {}, page_table, shift, num_pages};
+    swa_status st = ctl(&a.ctl);
+    if (st != SWA_OK) return st;
+    return from_cuda(swa::launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || W < 1 || Hq % Hkv) return 0;
@@ -360,10 +399,12 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
 
 namespace {
 
-// swa_decode and swa_decode_sinks (n_sink = 0: no sinks).
+// swa_decode, swa_decode_sinks (n_sink = 0: no sinks) and swa_decode_paged
+// (page_table not null: k_cache / v_cache are page pools).
 swa_status decode_impl(const void *q, const void *k_cache, const void *v_cache, const void *k_sink,
                        const void *v_sink, int n_sink, void *o, float *lse, const int32_t *pos, int B, int Hq, int Hkv,
-                       int d, int W, float scale, swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream)
+                       int d, int W, float scale, swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream,
+                       const int32_t *page_table = nullptr, int page_size = 0, int num_pages = 0)
 {
     if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
     if (n_sink < 0) return SWA_ERR_INVALID_ARG;
@@ -388,6 +429,12 @@ swa_status decode_impl(const void *q, const void *k_cache, const void *v_cache, 
     if (n_sink > 0) {
         if (!k_sink || !v_sink || !aligned(k_sink, 16) || !aligned(v_sink, 16)) return SWA_ERR_INVALID_ARG;
         a.ks = k_sink; a.vs = v_sink; a.n_sink = n_sink;
+    }
+    if (page_table) {
+        if (!aligned(page_table, 4)) return SWA_ERR_INVALID_ARG;
+        a.ptable = page_table;
+        a.page_shift = page_shift_of(page_size, W);
+        a.num_pages = num_pages;
     }
     swa_status st = ctl(&a.ctl);
     if (st != SWA_OK) return st;
@@ -417,6 +464,18 @@ swa_status swa_decode_sinks(const void *q, const void *k_cache, const void *v_ca
                        workspace, workspace_bytes, stream);
 }
 
+swa_status swa_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *page_table,
+                            void *o, float *lse, const int32_t *pos, int B, int Hq, int Hkv, int d, int W,
+                            int page_size, int num_pages, float scale, swa_dtype dt, void *workspace,
+                            size_t workspace_bytes, void *stream)
+{
+    SWA_NVTX_RANGE("swa_decode_paged");
+    if (W < 1 || num_pages < 1 || page_shift_of(page_size, W) < 0) return SWA_ERR_INVALID_ARG;
+    if (B > 0 && !page_table) return SWA_ERR_INVALID_ARG;
+    return decode_impl(q, k_pages, v_pages, nullptr, nullptr, 0, o, lse, pos, B, Hq, Hkv, d, W, scale, dt, workspace,
+                       workspace_bytes, stream, B > 0 ? page_table : nullptr, page_size, num_pages);
+}
+
 swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric, const int32_t *global_idx, int g,
                            void *stream)
 {
@@ -443,6 +502,7 @@ swa_status swa_get_device_status(void *stream)
     if (cudaMemcpyFromSymbol(&v, g_swa_status, sizeof(int)) != cudaSuccess) return SWA_ERR_CUDA;
     if (cudaMemcpyToSymbol(g_swa_status, &zero, sizeof(int)) != cudaSuccess) return SWA_ERR_CUDA;
     if (v >= SWA_STATUS_TIMEOUT) return SWA_ERR_TIMEOUT;
+    if (v == SWA_STATUS_DEBUG_CHECK) return SWA_ERR_INTERNAL;
     if (v == SWA_STATUS_BAD_INPUT) return SWA_ERR_INVALID_ARG;
     return SWA_OK;
 }

@@ -21,7 +21,24 @@ struct SwaNvtxRange {
 // Device status word values (ordered: the worst one wins via atomicMax).
 #define SWA_STATUS_OK 0
 #define SWA_STATUS_BAD_INPUT 1
+#define SWA_STATUS_DEBUG_CHECK 2
 #define SWA_STATUS_TIMEOUT 4
+
+// Device-side consistency checks of tile, row and slot indices, compiled in
+// only by the debug build (-DSWA_DEBUG, libswa_debug.so).  A failed check
+// records SWA_STATUS_DEBUG_CHECK in the status word (read by
+// swa_get_device_status as SWA_ERR_INTERNAL); it never traps.  In the release
+// build the checks compile to nothing.
+#ifdef SWA_DEBUG
+#define SWA_DCHECK(cond, status)                                                                                      \
+    do {                                                                                                              \
+        if (!(cond)) atomicMax((status), SWA_STATUS_DEBUG_CHECK);                                                     \
+    } while (0)
+#else
+#define SWA_DCHECK(cond, status)                                                                                      \
+    do {                                                                                                              \
+    } while (0)
+#endif
 
 namespace swa {
 
@@ -105,12 +122,18 @@ cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const Rin
 bool prefill_narrow_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s);
 
+// Band prefill with 128-key tiles and the two query tiles in alternation (no
+// global keys, sinks, ring or packed sequences), d = 64 or 128.
+bool prefill_pp_applies(int d, const TcPrefillArgs &a);
+cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s);
+
 // Packed variable-length sequences (causal band mode): q/k/v/o are
 // [total,H,d] (TcPrefillArgs.T = total, B = number of sequences) and
 // sequence b holds rows cu[b] .. cu[b+1]-1, none longer than max_len.
 struct VarlenArgs {
     const int32_t *cu;        // device [B+1]
     int max_len;
+    const int32_t *wseq;      // device [B]: window of each sequence, or null (TcPrefillArgs.left for all)
 };
 cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s);
 
@@ -132,9 +155,11 @@ struct F32PrefillArgs {
     int W_ring;
     DeviceCtl ctl;
     // packed sequences (B == 1, T = total rows): sequence s holds rows
-    // cu[s] .. cu[s+1]-1 (null: one sequence per batch row)
+    // cu[s] .. cu[s+1]-1 (null: one sequence per batch row), with window
+    // wseq[s] when wseq is not null (left = wseq[s]-1 instead of `left`)
     const int32_t *cu;
     int nseq;
+    const int32_t *wseq;
 };
 cudaError_t launch_prefill_f32(const F32PrefillArgs &a, cudaStream_t s);
 
@@ -152,7 +177,19 @@ struct DecodeArgs {
     // 0..n_sink-1 (n_sink = 0: none)
     const void *ks, *vs;
     int n_sink;
+    // paged ring (ptable not null): kc / vc are pools [num_pages,Hkv,P,d]
+    // with P = 2^page_shift; ring slot s of sequence b is row s mod P of
+    // page ptable[b*(W/P) + s/P]
+    const int32_t *ptable;
+    int page_shift, num_pages;
+    // set by launch_decode: the splits of a (sequence, kv head) form one
+    // thread-block cluster and merge through distributed shared memory
+    int cluster;
 };
+// Splits per (sequence, kv head); up to kClusterSplits of them merge inside
+// one thread-block cluster (no workspace), more need the workspace and a
+// combine launch.
+constexpr int kClusterSplits = 8;
 int decode_splits(int B, int Hq, int Hkv, int d, int W);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s);
@@ -165,6 +202,9 @@ struct AppendArgs {
     int B, n, Hkv, W;
     int row_bytes;            // d * element size
     DeviceCtl ctl;
+    // paged ring, as in DecodeArgs (null: dense [B,Hkv,W,d] caches)
+    const int32_t *ptable;
+    int page_shift, num_pages;
 };
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s);
 

@@ -51,7 +51,8 @@ typedef enum {
     SWA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0 ... */
     SWA_ERR_UNSUPPORTED = 2, /* valid request the library has no kernel for (e.g. d) */
     SWA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
-    SWA_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired; its outputs are invalid */
+    SWA_ERR_TIMEOUT = 4,     /* a kernel's bounded wait expired; its outputs are invalid */
+    SWA_ERR_INTERNAL = 5     /* debug build only: a device-side index check failed */
 } swa_status;
 
 typedef enum {
@@ -91,20 +92,30 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
 
 /*
  * Causal sliding-window prefill over packed sequences of different lengths
- * (variable-length batches): every sequence is its own causal prefill
- * (robocikowo.com opening definition); no row sees another sequence.
+ * (variable-length batches), each with its own window if asked: every
+ * sequence is its own causal prefill (robocikowo.com opening definition) and
+ * no row sees another sequence.  Windows may differ from sequence to sequence
+ * the way local layers of different models differ (Ultralytics glossary,
+ * section on alternating local and global layers: 4,096 tokens in Gemma 2,
+ * 1,024 in Gemma 3).
  *   q, o : [total,Hq,d]   k, v : [total,Hkv,d]   (rows of all sequences, one
  *          after the other)
  *   cu_seqlens : device int32 [nseq+1]: sequence s holds rows cu[s] ..
  *          cu[s+1]-1; cu[0] = 0, non-decreasing, cu[nseq] = total, each
  *          length <= max_seqlen (an entry breaking this makes its sequence
  *          empty and records SWA_ERR_INVALID_ARG in the device status word)
+ *   windows : nullable device int32 [nseq]: sequence s uses window
+ *          windows[s] >= 1 (an entry below 1 leaves that sequence's rows
+ *          untouched and records SWA_ERR_INVALID_ARG in the device status
+ *          word); NULL: every sequence uses W
  *   lse  : nullable fp32 [Hq,total]
- *   0 <= max_seqlen <= total; other arguments as swa_prefill.
+ *   0 <= max_seqlen <= total; W >= 1 even when `windows` is given; other
+ *   arguments as swa_prefill.
  */
 swa_status swa_prefill_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
-                              const int32_t *cu_seqlens, int nseq, int total, int max_seqlen,
-                              int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *stream);
+                              const int32_t *cu_seqlens, const int32_t *windows, int nseq, int total,
+                              int max_seqlen, int Hq, int Hkv, int d, int W, float scale, swa_dtype dt,
+                              void *stream);
 
 /*
  * Dilated sliding-window prefill (aivaro.ru section 4.2: instead of all
@@ -188,6 +199,32 @@ swa_status swa_cache_append(void *k_cache, void *v_cache, const void *k_new, con
                             const int32_t *pos, int32_t *slot_out,
                             int B, int n, int Hkv, int d, int W, swa_dtype dt, void *stream);
 
+/*
+ * Paged ring caches.  The W slots of each sequence's ring need not be one
+ * contiguous [W,d] block per kv head: they can live in W/P pages of P slots
+ * taken, in any order, from a pool shared by all sequences, the way a serving
+ * engine hands out fixed-size cache blocks.  The ring itself is unchanged:
+ * position i is ring slot i mod W (Ultralytics ring-buffer paragraph), and a
+ * sequence never needs more than W slots (dupenodi.dev, check-yourself
+ * question 1); the page table only says where each group of P slots is.
+ *   k_pages, v_pages : pools [num_pages,Hkv,P,d] (P = page_size)
+ *   page_table       : device int32 [B, W/P]: ring slot s of sequence b is
+ *                      row s mod P of page page_table[b*(W/P) + s/P]; an
+ *                      entry outside [0,num_pages) is recorded as
+ *                      SWA_ERR_INVALID_ARG in the device status word (append:
+ *                      that token is not written; decode: page 0 is read
+ *                      instead and the output is invalid)
+ *   page_size        : a power of two that divides W
+ * Pages of different sequences must not overlap.
+ */
+
+/* swa_cache_append into a paged ring; arguments as swa_cache_append, with
+ * the pools, page_table, page_size and num_pages as above. */
+swa_status swa_cache_append_paged(void *k_pages, void *v_pages, const void *k_new, const void *v_new,
+                                  const int32_t *pos, const int32_t *page_table, int32_t *slot_out,
+                                  int B, int n, int Hkv, int d, int W, int page_size, int num_pages,
+                                  swa_dtype dt, void *stream);
+
 /* Bytes of scratch swa_decode needs for these sizes (0 means none). */
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 
@@ -208,6 +245,17 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 swa_status swa_decode(const void *q, const void *k_cache, const void *v_cache, void *o, float *lse,
                       const int32_t *pos, int B, int Hq, int Hkv, int d, int W, float scale,
                       swa_dtype dt, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * swa_decode over a paged ring (see swa_cache_append_paged): the same step,
+ * the keys of ring slots 0 .. min(pos[b]+1,W)-1 read through page_table.
+ * The workspace is sized by swa_decode_workspace_bytes with the same B, Hq,
+ * Hkv, d, W.
+ */
+swa_status swa_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *page_table,
+                            void *o, float *lse, const int32_t *pos, int B, int Hq, int Hkv, int d, int W,
+                            int page_size, int num_pages, float scale, swa_dtype dt, void *workspace,
+                            size_t workspace_bytes, void *stream);
 
 /*
  * One decode step over the ring plus attention sinks (Ultralytics glossary,
@@ -267,7 +315,9 @@ swa_status swa_mask_export(uint8_t *mask, int T, int W, int symmetric,
 /*
  * Synchronises `stream`, then reads and clears the current device's status
  * word.  Returns SWA_ERR_TIMEOUT if a kernel gave up on a bounded wait since
- * the last call, SWA_ERR_INVALID_ARG if a kernel met a bad device-side input,
+ * the last call, SWA_ERR_INTERNAL if (debug build, libswa_debug.so, compiled
+ * with -DSWA_DEBUG) a kernel's check of its own tile, row or slot indices
+ * failed, SWA_ERR_INVALID_ARG if a kernel met a bad device-side input,
  * SWA_ERR_CUDA if synchronising failed, else SWA_OK.
  */
 swa_status swa_get_device_status(void *stream);

@@ -46,6 +46,7 @@ def test_exported_symbols_are_c_linkage():
 def test_status_strings(lib):
     assert swa.swa_status_string(0) == "ok"
     assert swa.swa_status_string(4) == "device wait timed out"
+    assert swa.swa_status_string(5) == "device consistency check failed (debug build)"
     assert swa.swa_status_string(99) == "unknown status"
 
 
@@ -129,15 +130,16 @@ def test_dilated_rejects(lib):
 
 def test_varlen_rejects(lib):
     f = lib.swa_prefill_varlen
-    call = lambda cu=FAKE, nseq=3, total=300, maxl=128, d=64: f(FAKE, FAKE, FAKE, FAKE, NULL, cu, nseq, total, maxl,
-                                                                8, 2, d, 64, 0.125, 1, NULL)
+    call = lambda cu=FAKE, nseq=3, total=300, maxl=128, d=64, win=NULL: f(FAKE, FAKE, FAKE, FAKE, NULL, cu, win, nseq,
+                                                                          total, maxl, 8, 2, d, 64, 0.125, 1, NULL)
     assert call(cu=NULL) == 1
     assert call(cu=ctypes.c_void_p((1 << 20) + 2)) == 1
     assert call(nseq=-1) == 1
     assert call(maxl=301) == 1
     assert call(d=48) == 2
+    assert call(win=ctypes.c_void_p((1 << 20) + 2)) == 1     # int32 windows need 4-byte alignment
     assert call(nseq=0, cu=NULL) == 0
-    assert f(NULL, NULL, NULL, NULL, NULL, NULL, 2, 0, 0, 8, 2, 64, 64, 0.125, 1, NULL) == 0   # no rows
+    assert f(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 2, 0, 0, 8, 2, 64, 64, 0.125, 1, NULL) == 0   # no rows
 
 
 def test_append_rejects(lib):
@@ -151,9 +153,9 @@ def test_append_rejects(lib):
 
 def test_decode_rejects(lib):
     f = lib.swa_decode
-    need = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
+    need = lib.swa_decode_workspace_bytes(2, 32, 8, 128, 4096)     # 32 splits: beyond one cluster
     assert need > 0
-    args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, vc=FAKE, o=FAKE, lse=NULL, pos=FAKE, B=64, Hq=32,
+    args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, vc=FAKE, o=FAKE, lse=NULL, pos=FAKE, B=2, Hq=32,
                                   Hkv=8, d=128, W=4096, scale=0.088, dt=1, ws=FAKE, wsb=need), **kw)
     call = lambda a: f(a["q"], a["kc"], a["vc"], a["o"], a["lse"], a["pos"], a["B"], a["Hq"], a["Hkv"],
                        a["d"], a["W"], a["scale"], a["dt"], a["ws"], a["wsb"], NULL)
@@ -180,7 +182,39 @@ def test_debug_hook_rejects_bad_limits(lib):
 
 
 def test_workspace_sizes(lib):
-    # no workspace when one split suffices; otherwise sized for [B,Hq,S,d+2] fp32
-    big = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
-    assert big % (64 * 32 * 130 * 4) == 0
+    # no workspace when one split suffices or the splits (at most 8) merge
+    # inside one thread-block cluster; otherwise [B,Hq,S,d+2] fp32
+    assert lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096) == 0      # 8 splits: one cluster
+    assert lib.swa_decode_workspace_bytes(2, 32, 8, 128, 4096) == 2 * 32 * 32 * 130 * 4   # 32 splits
+    assert lib.swa_decode_workspace_bytes(5, 32, 8, 128, 300) == 0        # one split
     assert lib.swa_decode_workspace_bytes(0, 32, 8, 128, 4096) == 0
+
+
+def test_paged_rejects(lib):
+    f = lib.swa_cache_append_paged
+    call = lambda tbl=FAKE, P=16, W=64, npg=8, d=64, pos=FAKE: f(FAKE, FAKE, FAKE, FAKE, pos, tbl, NULL, 2, 1, 2, d,
+                                                                 W, P, npg, 1, NULL)
+    assert call(tbl=NULL) == 1
+    assert call(P=12) == 1          # not a power of two
+    assert call(P=128) == 1         # does not divide W
+    assert call(P=0) == 1
+    assert call(npg=0) == 1
+    assert call(d=4) == 2           # 8-byte rows
+    assert call(tbl=ctypes.c_void_p((1 << 20) + 2)) == 1
+    g = lib.swa_decode_paged
+    need = lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096)
+    dcall = lambda tbl=FAKE, P=16, npg=16384, B=64: g(FAKE, FAKE, FAKE, tbl, FAKE, NULL, FAKE, B, 32, 8, 128, 4096,
+                                                      P, npg, 0.088, 1, FAKE, need, NULL)
+    assert dcall(tbl=NULL) == 1
+    assert dcall(P=24) == 1
+    assert dcall(npg=0) == 1
+    assert dcall(B=0, tbl=NULL) == 0
+
+
+def test_debug_build_exports_the_same_calls():
+    import subprocess
+    path = swa_build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    names = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in names, name
