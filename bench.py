@@ -391,7 +391,7 @@ def tinymistral_arm(swa, dev, args):
     nbytes = w.B * w.T * (2 * w.Hq + 2 * w.Hkv) * w.d * 2
     times = []
     for i in range(args.warmup + max(10, args.steps // 2)):
-        torch.sum(flush, out=sink)       # read sweep: evicts L2, leaves clean lines
+        torch.sum(flush, dim=0, out=sink)   # read sweep: evicts L2, leaves clean lines
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W, o=o)

@@ -276,7 +276,7 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
 }
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(PP_THREADS, 1)
     swa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                           const TcPrefillArgs a)
@@ -602,18 +602,22 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, cudaStream_t s)
 
 }  // namespace
 
+// Measured on B200 against the 64-key band kernel (same process, same
+// inputs): d = 128, causal W = 4096: 2.32 against 2.67 ms (Mistral-7B
+// prefill) and 0.48 against 0.55 ms at T = 8192; d = 128, W = 512: 0.32
+// against 0.31 ms; d = 64, W = 1024: equal; symmetric d = 64, W = 512: 0.255
+// against 0.225 ms.  So it takes the plain band prefill at d = 128 with a
+// window of at least 1024 keys, where each CTA streams enough key tiles for
+// the alternation of its two query tiles to pay.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a)
 {
-    return (d == 64 || d == 128) && a.gidx == nullptr && a.g == 0;
+    return d == 128 && a.gidx == nullptr && a.g == 0 && a.left + a.right + 1 >= 1024;
 }
 
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s)
 {
-    switch (d) {
-    case 64: return launch_pp_d<64>(a, s);
-    case 128: return launch_pp_d<128>(a, s);
-    default: return cudaErrorInvalidValue;
-    }
+    if (!prefill_pp_applies(d, a)) return cudaErrorInvalidValue;
+    return launch_pp_d<128>(a, s);
 }
 
 }  // namespace swa

@@ -126,6 +126,17 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Contiguous bulk copy global -> this CTA's shared memory, completion counted
+// on `bar` in bytes.  Both addresses 16-byte aligned, bytes a multiple of 16.
+// No multicast: the destination is this CTA's own shared memory.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // 4-D tiled store shared -> global (rows outside the tensor are clipped).
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int c0, int c1, int c2,
                                              int c3)
@@ -143,42 +154,6 @@ __device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bu
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// -------------------------------------------------------------- clusters --
-
-// This CTA's rank in its thread-block cluster.
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Every thread of every CTA of the cluster arrives, then waits for all: the
-// release/acquire pair orders shared-memory writes before it with the
-// distributed shared-memory reads of other CTAs after it.  A hardware barrier
-// (like __syncthreads), not a spin loop: every thread of the cluster must
-// reach it.
-__device__ __forceinline__ void cluster_sync()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address, in the cluster's shared window, of the same variable `p` in the
-// shared memory of CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t cluster_peer_addr(const void *p, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
 }
 
 // --------------------------------------------------------------- tcgen05 --

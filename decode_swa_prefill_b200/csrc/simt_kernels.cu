@@ -268,25 +268,19 @@ __device__ __forceinline__ long long paged_row(const DecodeArgs &a, const int32_
 }
 
 // The end of a decode CTA: merge the warps' partials (running max m in log2
-// units, sum l, unnormalised accumulator) held in shared memory, then
-//  - one split: write o (and lse);
-//  - splits in one thread-block cluster (a.cluster): keep the CTA's merged
-//    partial in shared memory; after a cluster barrier each CTA of the
-//    cluster merges a 1/splits slice of the G*D outputs, reading every
-//    split's partial from its CTA's shared memory (distributed shared
-//    memory), and writes o; a second barrier keeps every CTA's shared memory
-//    alive until the others have read it.  No workspace, no second launch.
-//  - otherwise: write the split's partial to the workspace for
-//    decode_combine_kernel.
-// The LSE merge: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// units, sum l, unnormalised accumulator) held in shared memory, then write
+// o (and lse) when the (sequence, kv head) has one split, else the split's
+// partial for decode_combine_kernel.  (Merging the splits inside a
+// thread-block cluster through distributed shared memory instead measured
+// slower: 219-238 us against 189-195 us at the 64-sequence decode workload,
+// the cluster's CTAs being scheduled together and waiting for the slowest at
+// the merge.)
 template <typename T, int D, int G>
 __device__ __forceinline__ void decode_finish(const DecodeArgs &a, int b, int hk, int split,
                                               const float (*sm_m)[G], const float (*sm_l)[G],
                                               const float (*sm_acc)[G][D])
 {
-    __shared__ float cm[G], cl[G], co[G][D];   // this CTA's merged partial (cluster merge)
     const int Hq = a.Hq;
-    const bool cluster = a.cluster && a.splits > 1;
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int g = idx / D, e = idx % D;
         float M = -CUDART_INF_F;
@@ -306,12 +300,6 @@ __device__ __forceinline__ void decode_finish(const DecodeArgs &a, int b, int hk
             Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
             if (a.lse && e == 0)
                 a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
-        } else if (cluster) {
-            co[g][e] = O;
-            if (e == 0) {
-                cm[g] = M;
-                cl[g] = L;
-            }
         } else {
             float *part = a.partial + (((long long)b * Hq + h) * a.splits + split) * (D + 2);
             part[e] = O;
@@ -321,29 +309,6 @@ __device__ __forceinline__ void decode_finish(const DecodeArgs &a, int b, int hk
             }
         }
     }
-    if (!cluster) return;
-    cluster_sync();
-    const int S = a.splits;
-    const int per = G * D / S;               // outputs this CTA merges
-    const int r0 = (int)cluster_ctarank() * per;
-    for (int idx = r0 + threadIdx.x; idx < r0 + per; idx += blockDim.x) {
-        const int g = idx / D, e = idx % D;
-        float M = -CUDART_INF_F;
-        for (int q = 0; q < S; ++q) M = fmaxf(M, ld_cluster_f32(cluster_peer_addr(&cm[g], q)));
-        const float Mu = M == -CUDART_INF_F ? 0.f : M;
-        float L = 0.f, O = 0.f;
-        for (int q = 0; q < S; ++q) {
-            const float f = ex2_approx(ld_cluster_f32(cluster_peer_addr(&cm[g], q)) - Mu);
-            L += ld_cluster_f32(cluster_peer_addr(&cl[g], q)) * f;
-            O += ld_cluster_f32(cluster_peer_addr(&co[g][e], q)) * f;
-        }
-        const int h = hk * G + g;
-        T *o = static_cast<T *>(a.o) + ((long long)b * Hq + h) * D;
-        Ld<T>::store(o + e, L > 0.f ? O / L : 0.f);
-        if (a.lse && e == 0)
-            a.lse[(long long)b * Hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
-    }
-    cluster_sync();
 }
 
 template <typename T, int D, int G, int SRC>
@@ -702,6 +667,223 @@ __global__ void __launch_bounds__(32 * DEC_WARPS)
     decode_finish<__nv_bfloat16, D, G>(a, b, hk, split, sm_m, sm_l, sm_acc);
 }
 
+// bf16 decode over a dense ring with the ring rows staged in shared memory.
+// Same CTAs (split, kv head, sequence), same slots per warp and the same
+// arithmetic as decode_bf16_kernel, but a fifth warp is a producer: each
+// stage of SS = 4*BATCH consecutive slots is one contiguous run of K rows and
+// one of V rows in the [B,Hkv,W,d] ring, copied with two cp.async.bulk
+// (no multicast) into a ring of BULK_NST stages; the four compute warps read
+// their rows from shared memory.  The bytes in flight per SM are then set by
+// the stages (up to 3 CTAs x 4 stages x 16 KB) instead of the compute warps'
+// registers (measured at the 64-sequence decode workload: 189 us back to
+// back against 195 us for decode_bf16_kernel).  Waits are bounded
+// (wait_bounded); on expiry the CTA records SWA_STATUS_TIMEOUT and the
+// producer lets its own copies land before the CTA exits.
+constexpr int BULK_NST = 4;
+constexpr int BULK_THREADS = 32 * (DEC_WARPS + 1);
+
+template <int D, int G>
+struct BulkCfg {
+    static constexpr int LPR = D / 8, RPW = 32 / LPR, NBL = LPR / G, BATCH = NBL * RPW;
+    static constexpr int SS = DEC_WARPS * BATCH;   // slots per stage
+    static constexpr int ROWB = D * 2;             // bytes per row
+    static constexpr int STAGE = SS * ROWB;        // bytes of K (or V) per stage
+    static constexpr int SMEM = 2 * BULK_NST * STAGE + 2 * BULK_NST * 8;
+    static constexpr bool OK = (G <= D / 8) && STAGE <= 8192;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(BULK_THREADS) decode_bulk_kernel(DecodeArgs a)
+{
+    using C = BulkCfg<D, G>;
+    constexpr int LPR = C::LPR, RPW = C::RPW, NBL = C::NBL, BATCH = C::BATCH;
+    extern __shared__ __align__(128) uint8_t dsm[];
+    uint8_t *sK = dsm;
+    uint8_t *sV = dsm + BULK_NST * C::STAGE;
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + 2 * BULK_NST * C::STAGE);
+    uint64_t *empty = full + BULK_NST;
+    __shared__ int abort_flag;
+    __shared__ float sm_m[DEC_WARPS][G], sm_l[DEC_WARPS][G];
+    __shared__ float sm_acc[DEC_WARPS][G][D];
+
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const long long p = a.pos[b];
+    if (p < 0 && threadIdx.x == 0 && split == 0 && hk == 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+    const int n_valid = p < 0 ? 0 : (int)(p + 1 < a.W ? p + 1 : a.W);
+    const int chunk = (a.W + a.splits - 1) / a.splits;
+    const int s_begin = split * chunk;
+    const int s_end = min(n_valid, s_begin + chunk);
+    const int n_it = s_end > s_begin ? (s_end - s_begin + C::SS - 1) / C::SS : 0;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < BULK_NST; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], DEC_WARPS);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    WaitCtl ctl{&abort_flag, a.ctl.status, a.ctl.limit_ns};
+
+    if (warp == DEC_WARPS) {
+        // ------------------------------------------------------ producer --
+        const long long ring0 = ((long long)b * a.Hkv + hk) * (long long)a.W * C::ROWB;
+        const uint8_t *kb = static_cast<const uint8_t *>(a.kc) + ring0;
+        const uint8_t *vb = static_cast<const uint8_t *>(a.vc) + ring0;
+        int iss[BULK_NST] = {};
+        bool ok = true;
+        for (int it = 0; it < n_it && ok; ++it) {
+            const int st = it % BULK_NST;
+            ok = warp_wait_bounded(&empty[st], ((it / BULK_NST) & 1) ^ 1, ctl);
+            if (!ok) break;
+            if (lane == 0) {
+                const int s0 = s_begin + it * C::SS;
+                const int rows = min(C::SS, s_end - s0);
+                SWA_DCHECK(s0 >= 0 && rows > 0 && s0 + rows <= a.W, a.ctl.status);
+                const uint32_t bytes = (uint32_t)(rows * C::ROWB);
+                mbar_expect_tx(&full[st], 2 * bytes);
+                bulk_load(sK + st * C::STAGE, kb + (long long)s0 * C::ROWB, bytes, &full[st]);
+                bulk_load(sV + st * C::STAGE, vb + (long long)s0 * C::ROWB, bytes, &full[st]);
+            }
+            iss[st]++;
+        }
+        if (!ok && lane == 0)
+            // let our own copies land before the CTA's shared memory goes away
+            for (int st = 0; st < BULK_NST; ++st) {
+                if (iss[st] == 0) continue;
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try_wait(&full[st], (iss[st] - 1) & 1))
+                    if (globaltimer() - t0 > a.ctl.limit_ns) break;
+            }
+    } else {
+        // ----------------------------------------------------- compute --
+        const int part = lane % LPR;        // which 8 elements of a row
+        const int rgrp = lane / LPR;        // which row of a warp load
+        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q) + ((long long)b * a.Hq + (long long)hk * G) * D;
+        uint4 q[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) q[g] = __ldg(reinterpret_cast<const uint4 *>(qb + g * D + part * 8));
+        float2 acc[G][4];
+        float m[G], l[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            m[g] = -CUDART_INF_F;
+            l[g] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
+        }
+        for (int it = 0; it < n_it; ++it) {
+            const int st = it % BULK_NST;
+            if (!warp_wait_bounded(&full[st], (it / BULK_NST) & 1, ctl)) break;
+            const int rows = min(C::SS, s_end - (s_begin + it * C::SS));
+            const int r0 = warp * BATCH;    // this warp's first row of the stage
+            if (r0 < rows) {
+                const uint8_t *kst = sK + st * C::STAGE + part * 16;
+                const uint8_t *vst = sV + st * C::STAGE + part * 16;
+                uint4 kr[NBL], vr[NBL];
+#pragma unroll
+                for (int n = 0; n < NBL; ++n) {
+                    const int r = min(r0 + n * RPW + rgrp, rows - 1); // clamp: masked below
+                    kr[n] = *reinterpret_cast<const uint4 *>(kst + r * C::ROWB);
+                    vr[n] = *reinterpret_cast<const uint4 *>(vst + r * C::ROWB);
+                }
+                float v[LPR];
+#pragma unroll
+                for (int n = 0; n < NBL; ++n)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float t = 0.f;
+                        t = dot2_bf16(q[g].x, kr[n].x, t);
+                        t = dot2_bf16(q[g].y, kr[n].y, t);
+                        t = dot2_bf16(q[g].z, kr[n].z, t);
+                        t = dot2_bf16(q[g].w, kr[n].w, t);
+                        v[n * G + g] = t;
+                    }
+#pragma unroll
+                for (int k = LPR / 2; k >= 1; k >>= 1) {
+                    const bool upper = (part & k) != 0;
+#pragma unroll
+                    for (int x = 0; x < k; ++x) {
+                        const float send = upper ? v[x] : v[x + k];
+                        const float keep = upper ? v[x + k] : v[x];
+                        v[x] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+                    }
+                }
+                const int my_n = part / G, my_g = part % G;
+                const float sc = (r0 + my_n * RPW + rgrp < rows) ? v[0] * a.scale_log2 : -CUDART_INF_F;
+                float bm = sc;
+#pragma unroll
+                for (int k = G; k < 32; k <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, k));
+                float m_old = m[0];
+#pragma unroll
+                for (int g = 1; g < G; ++g)
+                    if (my_g == g) m_old = m[g];
+                const float m_new = fmaxf(m_old, bm);
+                const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+                const float pr = ex2_approx(sc - m_use);
+                const float al = ex2_approx(m_old - m_use);
+                float ps = pr;
+#pragma unroll
+                for (int k = G; k < 32; k <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, k);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float alg = __shfl_sync(0xffffffffu, al, g);
+                    const float psg = __shfl_sync(0xffffffffu, ps, g);
+                    m[g] = __shfl_sync(0xffffffffu, m_new, g);
+                    l[g] = l[g] * alg + psg;
+                    const float2 a2 = make_float2(alg, alg);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[g][e] = mul2(acc[g][e], a2);
+                }
+#pragma unroll
+                for (int n = 0; n < NBL; ++n) {
+                    const float2 v0 = bf16x2_to_float2(vr[n].x), v1 = bf16x2_to_float2(vr[n].y);
+                    const float2 v2 = bf16x2_to_float2(vr[n].z), v3 = bf16x2_to_float2(vr[n].w);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float pn = __shfl_sync(0xffffffffu, pr, rgrp * LPR + n * G + g);
+                        const float2 p2 = make_float2(pn, pn);
+                        acc[g][0] = fma2(p2, v0, acc[g][0]);
+                        acc[g][1] = fma2(p2, v1, acc[g][1]);
+                        acc[g][2] = fma2(p2, v2, acc[g][2]);
+                        acc[g][3] = fma2(p2, v3, acc[g][3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // sum the row groups' accumulators (same softmax reference per head)
+#pragma unroll
+        for (int k = LPR; k < 32; k <<= 1)
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, k);
+                    acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, k);
+                }
+        if (lane == 0)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                sm_m[warp][g] = m[g];
+                sm_l[warp][g] = l[g];
+            }
+        if (rgrp == 0)
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sm_acc[warp][g][part * 8 + 2 * e] = acc[g][e].x;
+                    sm_acc[warp][g][part * 8 + 2 * e + 1] = acc[g][e].y;
+                }
+    }
+    __syncthreads();
+    decode_finish<__nv_bfloat16, D, G>(a, b, hk, split, sm_m, sm_l, sm_acc);
+}
+
 // LSE merge of the split partials: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
 template <typename T, int D>
 __global__ void decode_combine_kernel(DecodeArgs a)
@@ -723,24 +905,13 @@ __global__ void decode_combine_kernel(DecodeArgs a)
     if (a.lse && e == 0) a.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -CUDART_INF_F;
 }
 
-// One decode launch: grid (splits, Hkv, B), the splits of a (sequence, kv
-// head) as one cluster along x when they merge in the cluster.
+// One decode launch: grid (splits, Hkv, B).
 template <typename K>
-cudaError_t launch_decode_grid(K kernel, const DecodeArgs &a, cudaStream_t s)
+cudaError_t launch_decode_grid(K kernel, const DecodeArgs &a, cudaStream_t s, int threads = 32 * DEC_WARPS,
+                               int smem = 0)
 {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.splits, a.Hkv, a.B);
-    cfg.blockDim = dim3(32 * DEC_WARPS, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.cluster ? a.splits : 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, a);
+    kernel<<<dim3(a.splits, a.Hkv, a.B), threads, smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 template <typename T, int D, int G>
@@ -748,6 +919,22 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
     const int src = a.ptable ? SRC_PAGED : a.n_sink > 0 ? SRC_SINKS : SRC_RING;
     cudaError_t e;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && BulkCfg<D, G>::OK) {
+        if (src == SRC_RING) {
+            using C = BulkCfg<D, G>;
+            static DeviceOnce once;
+            e = once.get(
+                [&](int) {
+                    return cudaFuncSetAttribute(decode_bulk_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                C::SMEM);
+                },
+                nullptr);
+            if (e == cudaSuccess) e = launch_decode_grid(decode_bulk_kernel<D, G>, a, s, BULK_THREADS, C::SMEM);
+            if (e != cudaSuccess || a.splits == 1) return e;
+            decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
+            return cudaGetLastError();
+        }
+    }
     if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8) {
         if (src == SRC_PAGED) e = launch_decode_grid(decode_bf16_kernel<D, G, SRC_PAGED>, a, s);
         else if (src == SRC_SINKS) e = launch_decode_grid(decode_bf16_kernel<D, G, SRC_SINKS>, a, s);
@@ -757,7 +944,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
         else if (src == SRC_SINKS) e = launch_decode_grid(decode_kernel<T, D, G, SRC_SINKS>, a, s);
         else e = launch_decode_grid(decode_kernel<T, D, G, SRC_RING>, a, s);
     }
-    if (e != cudaSuccess || a.splits == 1 || a.cluster) return e;
+    if (e != cudaSuccess || a.splits == 1) return e;
     decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -820,14 +1007,12 @@ int decode_splits(int B, int Hq, int Hkv, int d, int W)
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W)
 {
     const int s = decode_splits(B, Hq, Hkv, d, W);
-    if (s <= kClusterSplits) return 0;   // one split, or merged inside a cluster
+    if (s <= 1) return 0;
     return (size_t)B * Hq * s * (d + 2) * sizeof(float);
 }
 
-cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &args, cudaStream_t s)
+cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s)
 {
-    DecodeArgs a = args;
-    a.cluster = a.splits > 1 && a.splits <= kClusterSplits;
     return dtype_bf16 ? launch_decode_d<__nv_bfloat16>(a, s) : launch_decode_d<float>(a, s);
 }
 

@@ -123,7 +123,8 @@ bool prefill_narrow_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s);
 
 // Band prefill with 128-key tiles and the two query tiles in alternation (no
-// global keys, sinks, ring or packed sequences), d = 64 or 128.
+// global keys, sinks, ring or packed sequences): d = 128 and windows of at
+// least 1024 keys.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s);
 
@@ -182,14 +183,7 @@ struct DecodeArgs {
     // page ptable[b*(W/P) + s/P]
     const int32_t *ptable;
     int page_shift, num_pages;
-    // set by launch_decode: the splits of a (sequence, kv head) form one
-    // thread-block cluster and merge through distributed shared memory
-    int cluster;
 };
-// Splits per (sequence, kv head); up to kClusterSplits of them merge inside
-// one thread-block cluster (no workspace), more need the workspace and a
-// combine launch.
-constexpr int kClusterSplits = 8;
 int decode_splits(int B, int Hq, int Hkv, int d, int W);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 cudaError_t launch_decode(int dtype_bf16, const DecodeArgs &a, cudaStream_t s);

@@ -45,7 +45,7 @@ def run_all():
     win = torch.tensor([17, 5, 200], dtype=torch.int32)
     check("prefill_varlen", swa.swa_prefill_varlen(d(qp), d(kp), d(vp), d(cu), d(win), 471),
           oracle.swa_prefill_varlen(qp, kp, vp, cu, [17, 5, 200])[0])
-    for B, W in ((3, 256), (2, 4096)):        # 2 splits in a cluster / 32 splits with a workspace
+    for B, W in ((3, 256), (2, 4096)):        # 2 and 32 splits
         qd, kc, vc, kn, vn, pos = wl.decode_inputs(B, 8, 2, 128, W, torch.bfloat16, seed=W, pos_lo=0, pos_hi=9000)
         kcd, vcd = d(kc), d(vc)
         swa.swa_cache_append(kcd, vcd, d(kn), d(vn), d(pos))
@@ -55,7 +55,7 @@ def run_all():
     kcd, vcd = d(kc), d(vc)
     swa.swa_cache_append(kcd, vcd, d(kn), d(vn), d(pos))
     rk2, rv2, _ = oracle.ring_append(kc, vc, kn, vn, pos)
-    check("decode cluster merge", swa.swa_decode(d(qd), kcd, vcd, d(pos)), oracle.swa_decode(qd, rk2, rv2, pos)[0])
+    check("decode 64 sequences", swa.swa_decode(d(qd), kcd, vcd, d(pos)), oracle.swa_decode(qd, rk2, rv2, pos)[0])
     check("decode_noalloc", swa.swa_decode_noalloc(d(qd), kcd, vcd, d(pos)), oracle.swa_decode(qd, rk2, rv2, pos)[0])
     # paged ring: pages of 16 slots in a scrambled order
     B, W, P = 3, 128, 16

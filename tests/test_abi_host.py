@@ -182,11 +182,10 @@ def test_debug_hook_rejects_bad_limits(lib):
 
 
 def test_workspace_sizes(lib):
-    # no workspace when one split suffices or the splits (at most 8) merge
-    # inside one thread-block cluster; otherwise [B,Hq,S,d+2] fp32
-    assert lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096) == 0      # 8 splits: one cluster
+    # no workspace when one split suffices; otherwise [B,Hq,S,d+2] fp32
+    assert lib.swa_decode_workspace_bytes(64, 32, 8, 128, 4096) == 64 * 32 * 8 * 130 * 4   # 8 splits
     assert lib.swa_decode_workspace_bytes(2, 32, 8, 128, 4096) == 2 * 32 * 32 * 130 * 4   # 32 splits
-    assert lib.swa_decode_workspace_bytes(5, 32, 8, 128, 300) == 0        # one split
+    assert lib.swa_decode_workspace_bytes(5, 32, 8, 128, 200) == 0        # one split (W < 256)
     assert lib.swa_decode_workspace_bytes(0, 32, 8, 128, 4096) == 0
 
 
