@@ -92,7 +92,7 @@ def load_peaks():
 
 # the sources each recorded kernel is built from
 KERNEL_SOURCES = {
-    "prefill_mistral": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
+    "prefill_mistral": ("prefill_pp.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
     "longformer": ("prefill_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
     "tinymistral": ("narrow_tc.cu", "ptx.cuh", "swa_internal.h", "tma_map.h"),
     "decode_mistral": ("simt_kernels.cu", "ptx.cuh", "swa_internal.h"),
@@ -353,11 +353,11 @@ def gpu_arm(args, world, rank, local):
                        "frac_of_hbm_peak": round(dec_gbs / peak_h, 4),
                        "frac_of_8tbs": round(dec_gbs / 8000.0, 4), "bytes": acc["bytes_dec"]},
         },
-        "roofline": {"kernel": "swa_prefill_tc_kernel<128> (Mistral-7B prefill)", "bound": "tensor",
+        "roofline": {"kernel": "swa_prefill_pp_kernel<128> (Mistral-7B prefill)", "bound": "tensor",
                      "achieved": round(pre_tf, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(pre_tf / peak_t, 4), "peak_source": peak_src + " bf16 burst",
                      "traffic": recorded_traffic("prefill_mistral")},
-        "roofline_decode": {"kernel": "decode_bf16_kernel<128,4> + combine", "bound": "hbm",
+        "roofline_decode": {"kernel": "decode_bulk_kernel<128,4> + decode_combine_kernel", "bound": "hbm",
                             "achieved": round(dec_gbs, 1), "peak": peak_h, "unit": "GB/s",
                             "frac": round(dec_gbs / peak_h, 4), "peak_source": peak_src + " copy",
                             "traffic": recorded_traffic("decode_mistral")},

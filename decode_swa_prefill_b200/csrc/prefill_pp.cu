@@ -185,76 +185,88 @@ __device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a)
     return w;
 }
 
-// Softmax of one 128-key tile for one row: scores -> running max / sum -> P
-// (bf16 pairs) over the first 64 columns of the tile's S columns, in two
-// passes over TMEM so that at most 64 scores are held in registers: the row
-// maximum from two 64-column halves, then per 32-column chunk the scores
-// again, their exponentials and the chunk's 16 columns of P.  P of chunk cc
-// lands in columns 16cc .. 16cc+15, which belong to S chunks already read
-// (cc/2 <= cc), so no score is overwritten before it is used.  FULL: every key
-// of the tile is visible to every row of the warp (no masking, all chunks
-// live), the common case, compiled without the masking branches.
+// Softmax of one 128-key tile for one row, one streaming pass over its four
+// 32-key chunks: chunk cc+1's TMEM load is in flight while chunk cc's scores
+// become exponentials and P (bf16 pairs in columns 16cc .. 16cc+15 of S,
+// inside S chunks already read), so at most 64 scores are held in registers
+// and one TMEM round trip per tile is exposed.  There is no separate maximum
+// pass: the running maximum m (log2 units) is raised when a chunk's own
+// maximum exceeds it by more than 2^8 -- after a row's first chunk that only
+// happens when its scores jump by that much -- by a whole number k of log2
+// units, and then l, this tile's sum so far and this tile's P chunks already
+// written are scaled by 2^-k, exactly (the caller scales the O row after the
+// previous PV).  P stays <= 256.
+// FULL: every key of the tile is visible to every row of the warp (no
+// masking, all chunks live), the common case, compiled without masking.
 template <bool FULL>
 __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c_hi, int col_lo, int col_hi,
                                                 float scale_log2, float &m, float &l, bool &rescale, float &alpha,
                                                 bool first)
 {
     auto live = [&](int cc) { return FULL || (cc >= c_lo && cc <= c_hi); };
-    auto mask32 = [&](float *v, int cc) {
-        if (!FULL) {
-            if (!live(cc)) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = -CUDART_INF_F;
-            } else {
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
+    float atot = 1.f;    // product of this tile's raises
+    auto chunk = [&](float *v, int cc) {
+        uint32_t pk[16];
+        if (live(cc)) {
+            if (!FULL) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int xx = cc * 32 + e;
                     if (xx < col_lo || xx > col_hi) v[e] = -CUDART_INF_F;
                 }
             }
-        }
-    };
-    // ---- pass 1: row maximum ----
-    float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+            float mx4[4];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        float sr[64];
-        if (live(2 * hh)) tmem_ld32(s_addr + hh * 64, sr);
-        if (live(2 * hh + 1)) tmem_ld32(s_addr + hh * 64 + 32, sr + 32);
-        tmem_ld_wait_dep(sr);
-        reg_fence32(sr + 32);
-        mask32(sr, 2 * hh);
-        mask32(sr + 32, 2 * hh + 1);
+            for (int j = 0; j < 4; ++j) mx4[j] = fmax3(v[j], v[4 + j], v[8 + j]);
 #pragma unroll
-        for (int e = 0; e + 8 <= 64; e += 8)
+            for (int e = 12; e + 8 <= 32; e += 8)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], sr[e + j], sr[e + 4 + j]);
-    }
-    const float mt = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
-    rescale = false;
-    alpha = 1.f;
-    if (mt > m + PP_RESCALE_LOG2) {
-        alpha = ex2_approx(m - mt);     // 0 when m was -inf
-        l *= alpha;
-        rescale = !first;
-        m = mt;
-    }
-    // ---- pass 2: exponentials and P, one 32-key chunk at a time ----
-    const float ref = (m == -CUDART_INF_F) ? 0.f : m;
-    const float2 sc2 = make_float2(scale_log2, scale_log2);
-    const float2 nr2 = make_float2(-ref, -ref);
-    float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
+                for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], v[e + j], v[e + 4 + j]);
 #pragma unroll
-    for (int cc = 0; cc < PP_BN / 32; ++cc) {
-        uint32_t pk[16];
-        if (live(cc)) {
-            float sr[32];
-            tmem_ld32(s_addr + cc * 32, sr);
-            tmem_ld_wait_dep(sr);
-            mask32(sr, cc);
+            for (int j = 0; j < 4; ++j) mx4[j] = fmaxf(mx4[j], v[28 + j]);
+            const float mc = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
+            const bool raise = mc > m + PP_RESCALE_LOG2;
+            float a = 1.f;
+            if (raise) {
+                if (m == -CUDART_INF_F) {
+                    a = 0.f;                // nothing accumulated yet
+                    m = mc;
+                } else {
+                    // a whole number k of log2 units: the factor 2^-k is exact,
+                    // so the bf16 P chunks rescaled below are not rounded twice
+                    const int k = (int)ceilf(mc - m);
+                    a = k < 126 ? __int_as_float((127 - k) << 23) : 0.f;
+                    m += (float)k;
+                }
+                l *= a;
+                acc2 = mul2(acc2, make_float2(a, a));
+                acc2b = mul2(acc2b, make_float2(a, a));
+                atot *= a;
+            }
+            // P chunks of this tile already in TMEM follow the new maximum
+            if (cc > 0 && __any_sync(0xffffffffu, raise)) {
+                tmem_st_wait();
+#pragma unroll 1
+                for (int pc = 0; pc < cc; ++pc) {
+                    float pv[16];
+                    tmem_ld16(s_addr + pc * 16, pv);
+                    tmem_ld_wait_dep16(pv);
+                    uint32_t pu[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint32_t w = __float_as_uint(pv[e]);
+                        pu[e] = pack_bf16x2(__uint_as_float(w << 16) * a, __uint_as_float(w & 0xffff0000u) * a);
+                    }
+                    tmem_st16u(s_addr + pc * 16, pu);
+                }
+            }
+            const float ref = (m == -CUDART_INF_F) ? 0.f : m;
+            const float2 nr2 = make_float2(-ref, -ref);
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-                float2 y = fma2(make_float2(sr[e], sr[e + 1]), sc2, nr2);
+                float2 y = fma2(make_float2(v[e], v[e + 1]), sc2, nr2);
                 if ((e / 2) % PP_POLY_EVERY == PP_POLY_EVERY - 1) {
                     y = exp2_poly2(y);
                 } else {
@@ -270,9 +282,24 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
             for (int j = 0; j < 16; ++j) pk[j] = 0u;
         }
         tmem_st16u(s_addr + cc * 16, pk);
-    }
+    };
+    float va[32], vb[32];
+    if (live(0)) tmem_ld32(s_addr, va);
+    tmem_ld_wait_dep(va);
+    if (live(1)) tmem_ld32(s_addr + 32, vb);
+    chunk(va, 0);
+    tmem_ld_wait_dep(vb);
+    if (live(2)) tmem_ld32(s_addr + 64, va);
+    chunk(vb, 1);
+    tmem_ld_wait_dep(va);
+    if (live(3)) tmem_ld32(s_addr + 96, vb);
+    chunk(va, 2);
+    tmem_ld_wait_dep(vb);
+    chunk(vb, 3);
     const float2 tot = add2(acc2, acc2b);
     l += tot.x + tot.y;
+    alpha = atot;
+    rescale = !first && atot != 1.f;
 }
 
 template <int D>

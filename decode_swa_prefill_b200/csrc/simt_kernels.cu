@@ -692,7 +692,7 @@ struct BulkCfg {
     static constexpr bool OK = (G <= D / 8) && STAGE <= 8192;
 };
 
-template <int D, int G>
+template <int D, int G, bool PAGED>
 __global__ void __launch_bounds__(BULK_THREADS) decode_bulk_kernel(DecodeArgs a)
 {
     using C = BulkCfg<D, G>;
@@ -729,9 +729,11 @@ __global__ void __launch_bounds__(BULK_THREADS) decode_bulk_kernel(DecodeArgs a)
 
     if (warp == DEC_WARPS) {
         // ------------------------------------------------------ producer --
-        const long long ring0 = ((long long)b * a.Hkv + hk) * (long long)a.W * C::ROWB;
+        const long long ring0 = PAGED ? 0 : ((long long)b * a.Hkv + hk) * (long long)a.W * C::ROWB;
         const uint8_t *kb = static_cast<const uint8_t *>(a.kc) + ring0;
         const uint8_t *vb = static_cast<const uint8_t *>(a.vc) + ring0;
+        const int32_t *tbl = PAGED ? a.ptable + (long long)b * (a.W >> a.page_shift) : nullptr;
+        bool bad_page = false;
         int iss[BULK_NST] = {};
         bool ok = true;
         for (int it = 0; it < n_it && ok; ++it) {
@@ -742,13 +744,29 @@ __global__ void __launch_bounds__(BULK_THREADS) decode_bulk_kernel(DecodeArgs a)
                 const int s0 = s_begin + it * C::SS;
                 const int rows = min(C::SS, s_end - s0);
                 SWA_DCHECK(s0 >= 0 && rows > 0 && s0 + rows <= a.W, a.ctl.status);
-                const uint32_t bytes = (uint32_t)(rows * C::ROWB);
-                mbar_expect_tx(&full[st], 2 * bytes);
-                bulk_load(sK + st * C::STAGE, kb + (long long)s0 * C::ROWB, bytes, &full[st]);
-                bulk_load(sV + st * C::STAGE, vb + (long long)s0 * C::ROWB, bytes, &full[st]);
+                mbar_expect_tx(&full[st], 2u * (uint32_t)(rows * C::ROWB));
+                if constexpr (PAGED) {
+                    // one copy per run of slots inside one page
+                    const int P = 1 << a.page_shift;
+                    for (int r = 0; r < rows;) {
+                        const int sl = s0 + r;
+                        const int n = min(P - (sl & (P - 1)), rows - r);
+                        const long long row = paged_row(a, tbl, hk, sl, &bad_page);
+                        bulk_load(sK + st * C::STAGE + r * C::ROWB, kb + row * C::ROWB, (uint32_t)(n * C::ROWB),
+                                  &full[st]);
+                        bulk_load(sV + st * C::STAGE + r * C::ROWB, vb + row * C::ROWB, (uint32_t)(n * C::ROWB),
+                                  &full[st]);
+                        r += n;
+                    }
+                } else {
+                    const uint32_t bytes = (uint32_t)(rows * C::ROWB);
+                    bulk_load(sK + st * C::STAGE, kb + (long long)s0 * C::ROWB, bytes, &full[st]);
+                    bulk_load(sV + st * C::STAGE, vb + (long long)s0 * C::ROWB, bytes, &full[st]);
+                }
             }
             iss[st]++;
         }
+        if (PAGED && bad_page) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
         if (!ok && lane == 0)
             // let our own copies land before the CTA's shared memory goes away
             for (int st = 0; st < BULK_NST; ++st) {
@@ -920,16 +938,21 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
     const int src = a.ptable ? SRC_PAGED : a.n_sink > 0 ? SRC_SINKS : SRC_RING;
     cudaError_t e;
     if constexpr (std::is_same<T, __nv_bfloat16>::value && BulkCfg<D, G>::OK) {
-        if (src == SRC_RING) {
+        if (src == SRC_RING || src == SRC_PAGED) {
             using C = BulkCfg<D, G>;
             static DeviceOnce once;
             e = once.get(
                 [&](int) {
-                    return cudaFuncSetAttribute(decode_bulk_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                C::SMEM);
+                    cudaError_t r = cudaFuncSetAttribute(decode_bulk_kernel<D, G, false>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+                    if (r != cudaSuccess) return r;
+                    return cudaFuncSetAttribute(decode_bulk_kernel<D, G, true>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
                 },
                 nullptr);
-            if (e == cudaSuccess) e = launch_decode_grid(decode_bulk_kernel<D, G>, a, s, BULK_THREADS, C::SMEM);
+            if (e == cudaSuccess)
+                e = src == SRC_PAGED ? launch_decode_grid(decode_bulk_kernel<D, G, true>, a, s, BULK_THREADS, C::SMEM)
+                                     : launch_decode_grid(decode_bulk_kernel<D, G, false>, a, s, BULK_THREADS, C::SMEM);
             if (e != cudaSuccess || a.splits == 1) return e;
             decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
             return cudaGetLastError();

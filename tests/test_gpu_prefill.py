@@ -67,6 +67,25 @@ def test_window_one_returns_v_exactly():
     assert torch.equal(o.cpu(), v.repeat_interleave(2, dim=2))
 
 
+@pytest.mark.parametrize("W", [64, 2048])
+def test_large_scores_exercise_every_rescale(W):
+    # q scaled by 4 (exact in bf16): log2-unit scores with a standard
+    # deviation near 6, so a row's running maximum is raised again and again,
+    # in a third of the rows also in the middle of a key tile -- the paths
+    # that rescale l, O and (in the 128-key kernel) the P chunks already
+    # written; W = 2048 at d = 128 runs the 128-key kernel, W = 64 the 64-key
+    # band kernel.  (Scaled by 8 or 16, the scores are so spread that bf16
+    # probabilities alone cost about 0.016 of max error, and every kernel
+    # here reaches 0.020-0.022.)
+    q, k, v = wl.prefill_inputs(1, 3000, 8, 2, 128, torch.bfloat16, seed=W)
+    q = q * 4
+    lse = torch.full((1, 8, 3000), float("nan"), device=dev())
+    o = swa.swa_prefill(q.to(dev()), k.to(dev()), v.to(dev()), W, lse=lse)
+    ref_o, ref_lse = oracle.swa_prefill(q, k, v, W)
+    assert max_err(o, ref_o) <= 2e-2
+    assert max_err(lse, ref_lse) <= 2e-2
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_masked_keys_weigh_exactly_zero(d):
     # W = 1: in each key tile every key but one is masked for a row.  Odd
