@@ -32,13 +32,16 @@
 // shared memory at the rate the tensor core consumes them (an N = 64 QK^T is
 // limited by shared-memory bandwidth instead).
 //
-// Softmax (one row per thread, 128 scores per tile): running maximum in log2
-// units, raised only when a tile's maximum exceeds it by more than 2^8 (P
-// stays <= 256 in bf16), which rescales l and the O row in TMEM after the
-// previous PV; -inf outside the window on edge tiles only; per warp, 32-key
-// chunks no row of the warp can see are skipped (their P is written as 0).
-// Three quarters of the exponentials run on the MUFU (ex2.approx), one
-// quarter as the range-reduced cubic exp2_poly2 on the FMA pipe.
+// Softmax (one row per thread, 128 scores per tile, one streaming pass over
+// four 32-key chunks): running maximum in log2 units, raised only when a
+// chunk's maximum exceeds it by more than 2^8 (P stays <= 256 in bf16), by a
+// whole power of two, which rescales l, the P chunks already written and the
+// O row in TMEM after the previous PV; -inf outside the window on edge tiles
+// only; per warp, 32-key chunks no row of the warp can see are skipped (their
+// P is written as 0).
+// Every exponential runs on the MUFU (ex2.approx): moving a quarter of them
+// to a cubic on the FMA pipe measured 2% slower here (the issue slots, not
+// the MUFU, are what the softmax runs short of).
 //
 // Every mbarrier wait is bounded (wait_bounded): on expiry the CTA records
 // SWA_STATUS_TIMEOUT, drains its own in-flight copies and MMAs with a second
@@ -59,7 +62,6 @@ constexpr int PP_BN = 128;               // keys per key tile
 constexpr int PP_NSTAGE = 2;             // K and V pipeline depth
 constexpr int PP_THREADS = 320;
 constexpr float PP_RESCALE_LOG2 = 8.0f;  // raise the running max only beyond 2^8
-constexpr int PP_POLY_EVERY = 4;         // every 4th pair of exponentials on the FMA pipe
 
 template <int D>
 struct PCfg {
@@ -207,72 +209,74 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
     const float2 sc2 = make_float2(scale_log2, scale_log2);
     float2 acc2 = make_float2(0.f, 0.f), acc2b = make_float2(0.f, 0.f);
     float atot = 1.f;    // product of this tile's raises
-    auto chunk = [&](float *v, int cc) {
+    // chunk maximum (log2 units, before the scale), -inf for a dead chunk;
+    // masked keys become -inf in place
+    auto cmax = [&](float *v, int cc) -> float {
+        if (!live(cc)) return -CUDART_INF_F;
+        if (!FULL) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int xx = cc * 32 + e;
+                if (xx < col_lo || xx > col_hi) v[e] = -CUDART_INF_F;
+            }
+        }
+        float mx4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx4[j] = fmax3(v[j], v[4 + j], v[8 + j]);
+#pragma unroll
+        for (int e = 12; e + 8 <= 32; e += 8)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], v[e + j], v[e + 4 + j]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx4[j] = fmaxf(mx4[j], v[28 + j]);
+        return fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+    };
+    // raise the running maximum for the pair of chunks from c0 on (maximum mc)
+    auto raise_to = [&](float mc, int c0) {
+        const bool raise = mc > m + PP_RESCALE_LOG2;
+        if (!__any_sync(0xffffffffu, raise)) return;
+        float a = 1.f;
+        if (raise) {
+            if (m == -CUDART_INF_F) {
+                a = 0.f;
+                m = mc;
+            } else {
+                const int k = (int)ceilf(mc - m);
+                a = k < 126 ? __int_as_float((127 - k) << 23) : 0.f;
+                m += (float)k;
+            }
+            l *= a;
+            acc2 = mul2(acc2, make_float2(a, a));
+            acc2b = mul2(acc2b, make_float2(a, a));
+            atot *= a;
+        }
+        if (c0 > 0) {
+            tmem_st_wait();
+#pragma unroll 1
+            for (int pc = 0; pc < c0; ++pc) {
+                float pv[16];
+                tmem_ld16(s_addr + pc * 16, pv);
+                tmem_ld_wait_dep16(pv);
+                uint32_t pu[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const uint32_t w = __float_as_uint(pv[e]);
+                    pu[e] = pack_bf16x2(__uint_as_float(w << 16) * a, __uint_as_float(w & 0xffff0000u) * a);
+                }
+                tmem_st16u(s_addr + pc * 16, pu);
+            }
+        }
+    };
+    auto exps = [&](float *v, int cc) {
         uint32_t pk[16];
         if (live(cc)) {
-            if (!FULL) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int xx = cc * 32 + e;
-                    if (xx < col_lo || xx > col_hi) v[e] = -CUDART_INF_F;
-                }
-            }
-            float mx4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) mx4[j] = fmax3(v[j], v[4 + j], v[8 + j]);
-#pragma unroll
-            for (int e = 12; e + 8 <= 32; e += 8)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) mx4[j] = fmax3(mx4[j], v[e + j], v[e + 4 + j]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) mx4[j] = fmaxf(mx4[j], v[28 + j]);
-            const float mc = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * scale_log2;
-            const bool raise = mc > m + PP_RESCALE_LOG2;
-            float a = 1.f;
-            if (raise) {
-                if (m == -CUDART_INF_F) {
-                    a = 0.f;                // nothing accumulated yet
-                    m = mc;
-                } else {
-                    // a whole number k of log2 units: the factor 2^-k is exact,
-                    // so the bf16 P chunks rescaled below are not rounded twice
-                    const int k = (int)ceilf(mc - m);
-                    a = k < 126 ? __int_as_float((127 - k) << 23) : 0.f;
-                    m += (float)k;
-                }
-                l *= a;
-                acc2 = mul2(acc2, make_float2(a, a));
-                acc2b = mul2(acc2b, make_float2(a, a));
-                atot *= a;
-            }
-            // P chunks of this tile already in TMEM follow the new maximum
-            if (cc > 0 && __any_sync(0xffffffffu, raise)) {
-                tmem_st_wait();
-#pragma unroll 1
-                for (int pc = 0; pc < cc; ++pc) {
-                    float pv[16];
-                    tmem_ld16(s_addr + pc * 16, pv);
-                    tmem_ld_wait_dep16(pv);
-                    uint32_t pu[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint32_t w = __float_as_uint(pv[e]);
-                        pu[e] = pack_bf16x2(__uint_as_float(w << 16) * a, __uint_as_float(w & 0xffff0000u) * a);
-                    }
-                    tmem_st16u(s_addr + pc * 16, pu);
-                }
-            }
             const float ref = (m == -CUDART_INF_F) ? 0.f : m;
             const float2 nr2 = make_float2(-ref, -ref);
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
                 float2 y = fma2(make_float2(v[e], v[e + 1]), sc2, nr2);
-                if ((e / 2) % PP_POLY_EVERY == PP_POLY_EVERY - 1) {
-                    y = exp2_poly2(y);
-                } else {
-                    y.x = ex2_approx(y.x);
-                    y.y = ex2_approx(y.y);
-                }
+                y.x = ex2_approx(y.x);
+                y.y = ex2_approx(y.y);
                 if (e & 2) acc2b = add2(acc2b, y);
                 else acc2 = add2(acc2, y);
                 pk[e / 2] = pack_bf16x2(y.x, y.y);
@@ -285,17 +289,19 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
     };
     float va[32], vb[32];
     if (live(0)) tmem_ld32(s_addr, va);
-    tmem_ld_wait_dep(va);
     if (live(1)) tmem_ld32(s_addr + 32, vb);
-    chunk(va, 0);
-    tmem_ld_wait_dep(vb);
-    if (live(2)) tmem_ld32(s_addr + 64, va);
-    chunk(vb, 1);
     tmem_ld_wait_dep(va);
+    reg_fence32(vb);
+    raise_to(fmaxf(cmax(va, 0), cmax(vb, 1)) * scale_log2, 0);
+    exps(va, 0);
+    if (live(2)) tmem_ld32(s_addr + 64, va);
+    exps(vb, 1);
     if (live(3)) tmem_ld32(s_addr + 96, vb);
-    chunk(va, 2);
-    tmem_ld_wait_dep(vb);
-    chunk(vb, 3);
+    tmem_ld_wait_dep(va);
+    reg_fence32(vb);
+    raise_to(fmaxf(cmax(va, 2), cmax(vb, 3)) * scale_log2, 2);
+    exps(va, 2);
+    exps(vb, 3);
     const float2 tot = add2(acc2, acc2b);
     l += tot.x + tot.y;
     alpha = atot;
@@ -454,14 +460,14 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             const int st = t % PP_NSTAGE;
             const bool more = t + 1 < w.n_tiles;
             ok = warp_wait_bounded(&bars->v_full[st], (t / PP_NSTAGE) & 1, ctl);
+            // the next K tile is waited for while tile A's softmax still runs
+            if (ok && more) ok = warp_wait_bounded(&bars->k_full[(t + 1) % PP_NSTAGE], ((t + 1) / PP_NSTAGE) & 1, ctl);
             if (!ok) break;
             // tile A: PV of key tile t, then QK^T of key tile t+1 into the
             // same S columns (issue order keeps them apart)
             if (pp_active(w.q[0], t)) ok = pv(0, t);
             if (!ok) break;
             if (more) {
-                ok = warp_wait_bounded(&bars->k_full[(t + 1) % PP_NSTAGE], ((t + 1) / PP_NSTAGE) & 1, ctl);
-                if (!ok) break;
                 tc_fence_after();
                 if (pp_active(w.q[0], t + 1)) qk(0, t + 1);
             }
