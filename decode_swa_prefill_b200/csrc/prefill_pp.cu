@@ -636,21 +636,22 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, cudaStream_t s)
 }  // namespace
 
 // Measured on B200 against the 64-key band kernel (same process, same
-// inputs): d = 128, causal W = 4096: 2.32 against 2.67 ms (Mistral-7B
-// prefill) and 0.48 against 0.55 ms at T = 8192; d = 128, W = 512: 0.32
-// against 0.31 ms; d = 64, W = 1024: equal; symmetric d = 64, W = 512: 0.255
-// against 0.225 ms.  So it takes the plain band prefill at d = 128 with a
-// window of at least 1024 keys, where each CTA streams enough key tiles for
-// the alternation of its two query tiles to pay.
+// inputs, T = 16384 unless stated, ms): d = 128, causal W = 256 / 512: 0.220 /
+// 0.278 against 0.238 / 0.312; W = 1024 equal; Mistral-7B prefill (W = 4096,
+// T = 32768) 2.007 against 2.666; d = 64, W = 256 / 512: 0.194 / 0.246
+// against 0.206 / 0.273; d = 32, W = 256 / 1024: 0.181 / 0.327 against 0.196
+// / 0.397; symmetric W = 512 (Longformer shapes, no globals) d = 64 0.207
+// against 0.225, d = 128 0.230 against 0.250.  So it takes every plain band
+// prefill (no global tokens) whose window spans at least 256 keys.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a)
 {
-    return d == 128 && a.gidx == nullptr && a.g == 0 && a.left + a.right + 1 >= 1024;
+    return (d == 32 || d == 64 || d == 128) && a.gidx == nullptr && a.g == 0 && a.left + a.right + 1 >= 256;
 }
 
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s)
 {
     if (!prefill_pp_applies(d, a)) return cudaErrorInvalidValue;
-    return launch_pp_d<128>(a, s);
+    return d == 128 ? launch_pp_d<128>(a, s) : d == 64 ? launch_pp_d<64>(a, s) : launch_pp_d<32>(a, s);
 }
 
 }  // namespace swa

@@ -1124,8 +1124,8 @@ cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArg
 // global rows only.
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
-    // a causal window of at most 64 keys: the single-pass kernel; wide
-    // windows at d = 128 without global keys: the 128-key kernel
+    // a causal window of at most 64 keys: the single-pass kernel; windows of
+    // 256 keys or more without global keys: the 128-key kernel
     if (mode == 0 && ring.pos == nullptr && prefill_narrow_applies(d, a)) return launch_prefill_narrow(d, a, s);
     if (mode == 0 && ring.pos == nullptr && prefill_pp_applies(d, a)) return launch_prefill_pp(d, a, s);
 

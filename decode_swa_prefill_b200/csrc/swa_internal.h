@@ -123,8 +123,8 @@ bool prefill_narrow_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s);
 
 // Band prefill with 128-key tiles and the two query tiles in alternation (no
-// global keys, sinks, ring or packed sequences): d = 128 and windows of at
-// least 1024 keys.
+// global keys, sinks, ring or packed sequences): d = 32, 64 or 128 and
+// windows of at least 256 keys.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s);
 
