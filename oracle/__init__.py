@@ -84,6 +84,9 @@ def _load():
         lib.oracle_swa_decode_paged.argtypes = [p, p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long,
                                                 c_long, c_long, c_double]
         lib.oracle_swa_decode_paged.restype = c_int
+        lib.oracle_swa_backward.argtypes = [p, p, p, p, p, p, p, c_long, c_long, c_long, c_long, c_long, c_long,
+                                            c_int, c_double, c_int]
+        lib.oracle_swa_backward.restype = c_int
         _lib = lib
     return _lib
 
@@ -419,3 +422,22 @@ def swa_prefill_varlen(q, k, v, cu_seqlens, W, scale=None, rows=None, nthreads=N
         return o, lse
     o, lse = _unflatten(o, lse, r, True, 1, total, Hq, d)
     return o[0], lse[0]
+
+
+def swa_backward(q, k, v, dout, W, symmetric=False, scale=None, nthreads=None):
+    """Gradients (dq [B,T,Hq,d], dk, dv [B,T,Hkv,d]) of the causal (or, with
+    symmetric=True, the |i-j| <= W//2) window prefill for the upstream
+    gradient dout [B,T,Hq,d].  The pages define only the forward pass; this is
+    its definition differentiated by the chain rule (see oracle.c)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
+    rc = _load().oracle_swa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     B, T, Hq, Hkv, d, W, 1 if symmetric else 0, float(scale),
+                                     nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_swa_backward: bad arguments")
+    return dq, dk, dv

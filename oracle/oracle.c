@@ -581,3 +581,117 @@ int oracle_swa_decode_sinks(const double *q, const double *kc, const double *vc,
     free(kr); free(vr); free(sc);
     return 0;
 }
+
+/* -------------------------------------------------------------- backward -- */
+
+/* Gradient of the sliding-window prefill (the causal or symmetric window of
+ * [P3 opening paragraph; P2 s.3, 4.1]) with respect to q, k and v, for an
+ * upstream gradient dO.  The pages define only the forward computation; this
+ * is that definition differentiated by the chain rule, row by row:
+ *   s_j  = scale q_i.k_j for j in the window,  p = softmax(s),  o_i = sum p_j v_j
+ *   dv_j += p_j dO_i
+ *   dp_j  = dO_i . v_j,   D = sum_j p_j dp_j  (= dO_i . o_i)
+ *   ds_j  = p_j (dp_j - D)
+ *   dq_i  = scale sum_j ds_j k_j,   dk_j += scale ds_j q_i
+ * Grouped-query heads: a kv head's dk, dv sum the rows of all its query heads.
+ * Every sum is an fp64 sum in index order.  Work is split over (b, kv head)
+ * so that each thread owns its dk, dv rows. */
+typedef struct {
+    const double *q, *k, *v, *dout;
+    double *dq, *dk, *dv;
+    long B, T, Hq, Hkv, d, W;
+    int mode;
+    double scale;
+    long next;
+    pthread_mutex_t mu;
+} backward_job;
+
+static void backward_group(backward_job *J, long b, long hk, long *keys, double *s, double *dp)
+{
+    const long T = J->T, d = J->d, Hq = J->Hq, Hkv = J->Hkv;
+    for (long h = 0; h < Hq; h++) {
+        if (h * Hkv / Hq != hk) continue;
+        for (long i = 0; i < T; i++) {
+            const double *qi = J->q + ((b * T + i) * Hq + h) * d;
+            const double *gi = J->dout + ((b * T + i) * Hq + h) * d;
+            double *dqi = J->dq + ((b * T + i) * Hq + h) * d;
+            long n = 0;
+            for (long j = 0; j < T; j++)
+                if (oracle_in_window(i, j, T, J->W, J->mode)) keys[n++] = j;
+            /* probabilities, two-pass */
+            double m = -INFINITY;
+            for (long c = 0; c < n; c++) {
+                const double *kj = J->k + ((b * T + keys[c]) * Hkv + hk) * d;
+                double acc = 0.0;
+                for (long e = 0; e < d; e++) acc += qi[e] * kj[e];
+                s[c] = J->scale * acc;
+                if (s[c] > m) m = s[c];
+            }
+            double l = 0.0;
+            for (long c = 0; c < n; c++) {
+                s[c] = exp(s[c] - m);
+                l += s[c];
+            }
+            for (long c = 0; c < n; c++) s[c] /= l;
+            /* dp_j = dO_i . v_j and D = sum p_j dp_j */
+            double D = 0.0;
+            for (long c = 0; c < n; c++) {
+                const double *vj = J->v + ((b * T + keys[c]) * Hkv + hk) * d;
+                double acc = 0.0;
+                for (long e = 0; e < d; e++) acc += gi[e] * vj[e];
+                dp[c] = acc;
+                D += s[c] * acc;
+            }
+            for (long e = 0; e < d; e++) dqi[e] = 0.0;
+            for (long c = 0; c < n; c++) {
+                const double ds = s[c] * (dp[c] - D);
+                const double *kj = J->k + ((b * T + keys[c]) * Hkv + hk) * d;
+                double *dkj = J->dk + ((b * T + keys[c]) * Hkv + hk) * d;
+                double *dvj = J->dv + ((b * T + keys[c]) * Hkv + hk) * d;
+                for (long e = 0; e < d; e++) {
+                    dqi[e] += J->scale * ds * kj[e];
+                    dkj[e] += J->scale * ds * qi[e];
+                    dvj[e] += s[c] * gi[e];
+                }
+            }
+        }
+    }
+}
+
+static void *backward_worker(void *arg)
+{
+    backward_job *J = (backward_job *)arg;
+    long *keys = malloc(sizeof(long) * (size_t)J->T);
+    double *s = malloc(sizeof(double) * (size_t)J->T);
+    double *dp = malloc(sizeof(double) * (size_t)J->T);
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        long u = J->next++;
+        pthread_mutex_unlock(&J->mu);
+        if (u >= J->B * J->Hkv) break;
+        backward_group(J, u / J->Hkv, u % J->Hkv, keys, s, dp);
+    }
+    free(keys); free(s); free(dp);
+    return NULL;
+}
+
+/* dq [B,T,Hq,d], dk and dv [B,T,Hkv,d] (all overwritten) for q, k, v, dout in
+ * the prefill layouts; mode ORACLE_CAUSAL or ORACLE_SYMMETRIC. */
+int oracle_swa_backward(const double *q, const double *k, const double *v, const double *dout, double *dq,
+                        double *dk, double *dv, long B, long T, long Hq, long Hkv, long d, long W, int mode,
+                        double scale, int nthreads)
+{
+    if (mode != ORACLE_CAUSAL && mode != ORACLE_SYMMETRIC) return -1;
+    memset(dk, 0, sizeof(double) * (size_t)(B * T * Hkv * d));
+    memset(dv, 0, sizeof(double) * (size_t)(B * T * Hkv * d));
+    backward_job J = {q, k, v, dout, dq, dk, dv, B, T, Hq, Hkv, d, W, mode, scale};
+    if (nthreads < 1) nthreads = 1;
+    J.next = 0;
+    pthread_mutex_init(&J.mu, NULL);
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; t++) pthread_create(&th[t], NULL, backward_worker, &J);
+    for (int t = 0; t < nthreads; t++) pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.mu);
+    return 0;
+}
