@@ -43,7 +43,7 @@ EXPORTED = [
     "swa_cache_append", "swa_decode_workspace_bytes",
     "swa_decode", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
     "swa_set_wait_limit_ns", "swa_status_string", "swa_decode_noalloc", "swa_cache_append_paged",
-    "swa_decode_paged",
+    "swa_decode_paged", "swa_prefill_backward", "swa_prefill_backward_workspace_bytes",
 ]
 
 _lib = None
@@ -81,6 +81,10 @@ def load():
     lib.swa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P]
     lib.swa_cache_append_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
     lib.swa_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P, ctypes.c_size_t, P]
+    lib.swa_prefill_backward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, P,
+                                         ctypes.c_size_t, P]
+    lib.swa_prefill_backward_workspace_bytes.argtypes = [I, I, I]
+    lib.swa_prefill_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.swa_mask_export.argtypes = [P, I, I, I, P, I, P]
     lib.swa_get_device_status.argtypes = [P]
     lib.swa_debug_expire_wait.argtypes = [I, P]
@@ -92,7 +96,7 @@ def load():
                  "swa_prefill_dilated", "swa_prefill_varlen",
                  "swa_cache_append", "swa_decode",
                  "swa_decode_noalloc", "swa_mask_export", "swa_get_device_status", "swa_debug_expire_wait",
-                 "swa_cache_append_paged", "swa_decode_paged"):
+                 "swa_cache_append_paged", "swa_decode_paged", "swa_prefill_backward"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -201,6 +205,37 @@ def swa_prefill_dilated(q, k, v, W, dil, symmetric=False, scale=None, o=None, ls
                                     _stream(stream))
     _check(st, "swa_prefill_dilated")
     return o
+
+
+def swa_prefill_backward_workspace_bytes(B, T, Hq):
+    return int(load().swa_prefill_backward_workspace_bytes(B, T, Hq))
+
+
+def swa_prefill_backward(q, k, v, o, lse, dout, W, symmetric=False, scale=None, dq=None, dk=None, dv=None,
+                         workspace=None, stream=None):
+    """Gradients of the window prefill (causal, or symmetric without
+    globals) for the upstream gradient dout: returns dq, dk, dv.  o and lse
+    are the forward call's outputs for the same q, k, v; the workspace (fp32
+    [B,Hq,T]) is allocated here when not given."""
+    _dev_contig(q, k, v, o, lse, dout, dq, dk, dv, workspace)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(k.shape == (B, T, Hkv, d) and v.shape == k.shape, "k/v shape")
+    _need(o.shape == q.shape and dout.shape == q.shape, "o/dout shape")
+    _need(lse.shape == (B, Hq, T) and lse.dtype == torch.float32, "lse must be fp32 [B,Hq,T]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = swa_prefill_backward_workspace_bytes(B, T, Hq)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = d ** -0.5 if scale is None else scale
+    st = load().swa_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                     _ptr(dv), int(bool(symmetric)), B, T, Hq, Hkv, d, W, float(scale),
+                                     _dtype_code(q), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "swa_prefill_backward")
+    return dq, dk, dv
 
 
 def swa_prefill_sinks(q, k, v, W, n_sink, scale=None, o=None, lse=None, stream=None):

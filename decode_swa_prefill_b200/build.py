@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libswa.so")
 DEBUG_LIB = os.path.join(HERE, "libswa_debug.so")
 SOURCES = ["swa_abi.cu", "prefill_tc.cu", "prefill_pp.cu", "narrow_tc.cu", "simt_kernels.cu", "decode_noalloc.cu",
-           "dilated.cu"]
+           "dilated.cu", "backward_tc.cu"]
 HEADERS = ["ptx.cuh", "swa_internal.h", "tma_map.h"]
 
 

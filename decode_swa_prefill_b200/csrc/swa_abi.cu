@@ -190,6 +190,48 @@ swa_status swa_prefill_global(const void *q, const void *k, const void *v, void 
     return from_cuda(swa::launch_prefill_tc(d, 0, a, swa::RingArgs{}, s));
 }
 
+size_t swa_prefill_backward_workspace_bytes(int B, int T, int Hq)
+{
+    if (B <= 0 || T <= 0 || Hq < 1) return 0;
+    return ((size_t)B * T * Hq * sizeof(float) + 255) & ~(size_t)255;
+}
+
+swa_status swa_prefill_backward(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                const void *dout, void *dq, void *dk, void *dv, int symmetric, int B, int T, int Hq,
+                                int Hkv, int d, int W, float scale, swa_dtype dt, void *workspace,
+                                size_t workspace_bytes, void *stream)
+{
+    SWA_NVTX_RANGE("swa_prefill_backward");
+    if (!valid_dtype(dt)) return SWA_ERR_INVALID_ARG;
+    if (symmetric != 0 && symmetric != 1) return SWA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
+    if (dt != SWA_DTYPE_BF16 || (d != 64 && d != 128)) return SWA_ERR_UNSUPPORTED;
+    if ((long long)B * T * Hq > (1LL << 31) || Hq > 65535 || B > 65535) return SWA_ERR_UNSUPPORTED;
+    if (B == 0 || T == 0) return SWA_OK;
+    const void *p16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+    for (const void *p : p16)
+        if (!p || !aligned(p, 16)) return SWA_ERR_INVALID_ARG;
+    if (!lse || !aligned(lse, 4)) return SWA_ERR_INVALID_ARG;
+    if (workspace_bytes < swa_prefill_backward_workspace_bytes(B, T, Hq)) return SWA_ERR_INVALID_ARG;
+    swa::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
+    a.delta = static_cast<float *>(workspace);
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv;
+    if (symmetric) {
+        a.left = a.right = W / 2 < T ? W / 2 : T;
+    } else {
+        a.left = W - 1 < T ? W - 1 : T;
+        a.right = 0;
+    }
+    a.scale = scale;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    swa_status st = ctl(&a.ctl);
+    if (st != SWA_OK) return st;
+    return from_cuda(swa::launch_prefill_backward(d, a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t swa_prefill_dilated_workspace_bytes(int B, int T, int Hq, int Hkv, int d, int dil, swa_dtype dt, int with_lse)
 {
     if (!valid_dtype(dt) || B <= 0 || T <= 0 || Hq < 1 || Hkv < 1 || d < 1 || dil <= 1) return 0;

@@ -122,6 +122,19 @@ cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const Rin
 bool prefill_narrow_applies(int d, const TcPrefillArgs &a);
 cudaError_t launch_prefill_narrow(int d, const TcPrefillArgs &a, cudaStream_t s);
 
+// ---- backward pass of the window prefill (bf16, d = 64 or 128) ----
+struct BwdArgs {
+    const void *q, *k, *v, *o, *dout;   // [B,T,Hq,d] / [B,T,Hkv,d]
+    const float *lse;                   // [B,Hq,T] natural log, from the forward pass
+    float *delta;                       // [B,Hq,T] scratch: dout_i . o_i
+    void *dq, *dk, *dv;                 // outputs, bf16
+    int B, T, Hq, Hkv;
+    int left, right;                    // window: keys i-left .. i+right
+    float scale, scale_log2;
+    DeviceCtl ctl;
+};
+cudaError_t launch_prefill_backward(int d, const BwdArgs &a, cudaStream_t s);
+
 // Band prefill with 128-key tiles and the two query tiles in alternation (no
 // global keys, sinks, ring or packed sequences): d = 32, 64 or 128 and
 // windows of at least 256 keys.

@@ -302,6 +302,30 @@ swa_status swa_decode_noalloc(const void *q, const void *k_cache, const void *v_
                               swa_dtype dt, void *stream);
 
 /*
+ * Backward pass of the window prefill: the gradients of swa_prefill
+ * (symmetric = 0) or of swa_prefill_global without globals (symmetric = 1)
+ * with respect to q, k and v, for an upstream gradient dout.  The pages
+ * define only the forward computation ("Sliding Window Attention",
+ * robocikowo.com, opening definition); this is its chain rule, with the
+ * probabilities recomputed from the forward pass's log-sum-exp:
+ *   p_ij = exp(scale q_i.k_j - lse_i) in the window, D_i = dout_i . o_i,
+ *   ds_ij = p_ij (dout_i.v_j - D_i), dq_i = scale sum_j ds_ij k_j,
+ *   dk_j = scale sum_i ds_ij q_i, dv_j = sum_i p_ij dout_i
+ * (a kv head's dk, dv sum over the query heads of its group).
+ *   q, o, dout, dq : [B,T,Hq,d]   k, v, dk, dv : [B,T,Hkv,d]   bf16
+ *   lse        : fp32 [B,Hq,T], the forward call's lse for the same inputs
+ *   workspace  : device scratch of swa_prefill_backward_workspace_bytes(...)
+ *                bytes, 16-byte aligned; calls sharing it must not overlap
+ *   bf16 only (SWA_ERR_UNSUPPORTED otherwise); d in {64, 128}; W >= 1;
+ *   other arguments as swa_prefill.  dq, dk, dv are overwritten.
+ */
+size_t swa_prefill_backward_workspace_bytes(int B, int T, int Hq);
+swa_status swa_prefill_backward(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                const void *dout, void *dq, void *dk, void *dv, int symmetric, int B, int T,
+                                int Hq, int Hkv, int d, int W, float scale, swa_dtype dt, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Debug export of the visibility mask, from the same device predicate the
  * prefill kernels apply (robocikowo.com binary-mask entry).
  *   mask : device uint8 [T,T], mask[i*T+j] = 1 when query i may see key j

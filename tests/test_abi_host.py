@@ -217,3 +217,21 @@ def test_debug_build_exports_the_same_calls():
     names = {line.split()[-1] for line in out.splitlines() if line.strip()}
     for name in declared_functions():
         assert name in names, name
+
+def test_backward_rejects(lib):
+    f = lib.swa_prefill_backward
+    need = lib.swa_prefill_backward_workspace_bytes(2, 300, 8)
+    assert need == (2 * 300 * 8 * 4 + 255) // 256 * 256
+    call = lambda sym=0, d=128, dt=1, ws=FAKE, wsb=need, lse=FAKE, W=64: f(FAKE, FAKE, FAKE, FAKE, lse, FAKE, FAKE,
+                                                                             FAKE, FAKE, sym, 2, 300, 8, 2, d, W,
+                                                                             0.088, dt, ws, wsb, NULL)
+    assert call(dt=0) == 2           # fp32: no backward kernel
+    assert call(d=32) == 2
+    assert call(sym=2) == 1
+    assert call(W=0) == 1
+    assert call(wsb=need - 1) == 1
+    assert call(ws=NULL) == 1
+    assert call(lse=NULL) == 1
+    assert call(lse=ctypes.c_void_p((1 << 20) + 2)) == 1
+    assert f(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 0, 300, 8, 2, 128, 64, 0.088, 1, NULL, 0,
+             NULL) == 0      # B == 0
