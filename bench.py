@@ -311,6 +311,7 @@ def gpu_arm(args, world, rank, local):
     extra, tiny_o = tinymistral_arm(swa, dev, args)
     toy, toy_o = toy_arm(swa, dev, args)
     chunk = chunk_arm(swa, dev, args)
+    backward = backward_arm(swa, dev, args, peaks)
     sinks = sinks_arm(swa, dev, args, load_peaks()[0])
     dilated = dilated_arm(swa, dev, args, load_peaks()[0])
     varlen = varlen_arm(swa, dev, args, load_peaks()[0])
@@ -345,6 +346,7 @@ def gpu_arm(args, world, rank, local):
             "tinymistral_prefill": extra,
             "toy_f32": toy,
             "chunk_prefill": chunk,
+            "prefill_backward": backward,
             "sinks": sinks,
             "dilated": dilated,
             "varlen": varlen,
@@ -457,6 +459,37 @@ def chunk_arm(swa, dev, args):
     tf = flops / (ms * 1e-3) / 1e12
     return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
             "flops": flops, "workload": w.name}
+
+
+def backward_arm(swa, dev, args, peaks):
+    """Backward pass of the Mistral-7B prefill (dq, dk, dv for a seeded
+    upstream gradient): not part of the step.  FLOPs: 5 matmuls of 2*d per
+    in-window pair (the recomputed Q K^T, dO V^T, P^T dO, dS^T Q, dS K), the
+    usual 2.5x of the forward's 4*d.  Inputs and outputs (1.3 GB) exceed L2."""
+    w = wl.MISTRAL_PREFILL
+    q, k, v = (t.to(dev) for t in wl.prefill_inputs(w.B, w.T, w.Hq, w.Hkv, w.d, w.dtype, w.seed))
+    g = torch.Generator().manual_seed(w.seed + 500)
+    dout = torch.randn(w.B, w.T, w.Hq, w.d, generator=g).to(w.dtype).to(dev)
+    lse = torch.empty(w.B, w.Hq, w.T, dtype=torch.float32, device=dev)
+    o = swa.swa_prefill(q, k, v, w.W, lse=lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(swa.swa_prefill_backward_workspace_bytes(w.B, w.T, w.Hq), dtype=torch.uint8, device=dev)
+    flops = causal_pairs(w.T, w.W) * w.B * w.Hq * 10 * w.d
+    times = []
+    for i in range(args.warmup + max(5, args.steps // 4)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        swa.swa_prefill_backward(q, k, v, o, lse, dout, w.W, dq=dq, dk=dk, dv=dv, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    assert swa.swa_get_device_status() == 0, "device status after the backward pass"
+    ms = sum(times) / len(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"tflops": round(tf, 2), "ms": round(ms, 4), "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+            "flops": flops, "workload": w.name + "_backward",
+            "kernels": "bwd_delta_kernel + bwd_dq_kernel<128> + bwd_dkdv_kernel<128>"}
 
 
 def dilated_pairs(T, W, dil, symmetric):
