@@ -878,6 +878,7 @@ PROFILE_CASES = {
     "tinymistral": (wl.TINYMISTRAL, {}),
     "chunk": (wl.MISTRAL_CHUNK, {}),
     "decode": (wl.MISTRAL_DECODE, {}),
+    "backward": (wl.MISTRAL_PREFILL, {"T": 8192}),
 }
 
 
@@ -891,8 +892,15 @@ def profile_case(name, launches):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     inp = {k: v.to(dev) for k, v in wl.make(w).items()}
+    if name == "backward":
+        lse = torch.empty(w.B, w.Hq, w.T, dtype=torch.float32, device=dev)
+        o = swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W, lse=lse)
+        dout = torch.randn(w.B, w.T, w.Hq, w.d, generator=torch.Generator().manual_seed(w.seed + 500)).to(w.dtype)
+        dout = dout.to(dev)
     for _ in range(launches):
-        if w.kind == "prefill":
+        if name == "backward":
+            swa.swa_prefill_backward(inp["q"], inp["k"], inp["v"], o, lse, dout, w.W)
+        elif w.kind == "prefill":
             swa.swa_prefill(inp["q"], inp["k"], inp["v"], w.W)
         elif w.kind == "prefill_global":
             swa.swa_prefill_global(inp["q"], inp["k"], inp["v"], inp["global_idx"], w.W)
