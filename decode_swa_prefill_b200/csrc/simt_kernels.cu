@@ -906,6 +906,10 @@ __global__ void __launch_bounds__(BULK_THREADS) decode_bulk_kernel(DecodeArgs a)
 template <typename T, int D>
 __global__ void decode_combine_kernel(DecodeArgs a)
 {
+    // launched as a programmatic dependent of the split kernel: its launch
+    // overlaps the split kernel's tail, and this wait returns once that
+    // kernel has completed and its partials are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int bh = blockIdx.x;
     const int e = threadIdx.x;
     const float *part = a.partial + (long long)bh * a.splits * (D + 2);
@@ -932,6 +936,24 @@ cudaError_t launch_decode_grid(K kernel, const DecodeArgs &a, cudaStream_t s, in
     return cudaGetLastError();
 }
 
+// The split merge, launched as a programmatic dependent of the split kernel
+// before it on the stream (its griddepcontrol.wait orders it after that
+// kernel's completion).
+template <typename T, int D>
+cudaError_t launch_combine(const DecodeArgs &a, cudaStream_t s)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.Hq);
+    cfg.blockDim = dim3(D);
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<T, D>, a);
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
 {
@@ -954,8 +976,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
                 e = src == SRC_PAGED ? launch_decode_grid(decode_bulk_kernel<D, G, true>, a, s, BULK_THREADS, C::SMEM)
                                      : launch_decode_grid(decode_bulk_kernel<D, G, false>, a, s, BULK_THREADS, C::SMEM);
             if (e != cudaSuccess || a.splits == 1) return e;
-            decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
-            return cudaGetLastError();
+            return launch_combine<T, D>(a, s);
         }
     }
     if constexpr (std::is_same<T, __nv_bfloat16>::value && G <= D / 8) {
@@ -968,8 +989,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s)
         else e = launch_decode_grid(decode_kernel<T, D, G, SRC_RING>, a, s);
     }
     if (e != cudaSuccess || a.splits == 1) return e;
-    decode_combine_kernel<T, D><<<a.B * a.Hq, D, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_combine<T, D>(a, s);
 }
 
 template <typename T, int D>
