@@ -50,6 +50,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "swa_internal.h"
 #include "tma_map.h"
@@ -104,6 +106,23 @@ __device__ __forceinline__ uint32_t pp_tile_offset(int r, int e, int ch_bytes)
     return ch * ch_bytes + r * C::RB + phys * 16;
 }
 
+// Producer-warp gather of a 128-key tile, one row at a time, into the
+// swizzled layout of a TMA tile load: 16-byte cp.async copies, all in flight
+// at once; row_src(r) gives key row r's source, or null for zeros.  All 32
+// lanes; returns once the copies have landed.
+template <int D, typename RowSrc>
+__device__ __forceinline__ void pp_gather_rows(uint8_t *dst, const __nv_bfloat16 *any_valid, int lane, RowSrc row_src)
+{
+    using C = PCfg<D>;
+    constexpr int GR = D / 8;   // 16-byte granules per row
+    for (int idx = lane; idx < PP_BN * GR; idx += 32) {
+        const int r = idx / GR, u = idx % GR;
+        const __nv_bfloat16 *src = row_src(r);
+        cp_async16(dst + pp_tile_offset<D>(r, u * 8, C::KCH), src ? src + u * 8 : any_valid, src ? 16u : 0u);
+    }
+    cp_async_wait_all();
+}
+
 struct PPBars {
     uint64_t q_full;
     uint64_t k_full[PP_NSTAGE];
@@ -138,6 +157,8 @@ struct PPWork {
     PPTile q[2];
     int j_lo;      // first key tile (absolute, 128-key units)
     int n_tiles;   // key tiles the CTA streams
+    long long p0;  // position of query row 0 (a chunk continuing a ring; else 0)
+    long long kend; // one past the last key position (p0 + T)
 };
 
 __device__ __forceinline__ bool pp_active(const PPTile &q, int t) { return q.active && t >= q.ts && t < q.te; }
@@ -145,7 +166,11 @@ __device__ __forceinline__ bool pp_active(const PPTile &q, int t) { return q.act
 // Units: pairs of query heads of one kv head (even group size) or pairs of
 // consecutive row tiles of one head; query tiles in descending order, so the
 // short CTAs at the start of a causal sequence run last and fill the tail.
-__device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a)
+// RING: the rows are a chunk of new tokens at positions pos[b] .. (a
+// negative entry is read as 0; the producer records it), and key tiles are
+// counted in absolute positions.
+template <bool RING>
+__device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const RingArgs &ring)
 {
     PPWork w;
     const int G = a.Hq / a.Hkv;
@@ -167,21 +192,27 @@ __device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a)
             if (qt < nqt) w.q[x] = PPTile{h, qt * PP_BM, min(PP_BM, a.T - qt * PP_BM), 0, 0, true};
         }
     }
-    int lo = a.T, hi = -1;
-    int lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
+    // positions: 64-bit only for a chunk continuing a ring
+    typedef typename std::conditional<RING, long long, int>::type kpos_t;
+    w.p0 = 0;
+    if constexpr (RING) w.p0 = max((long long)ring.pos[w.b], 0LL);
+    w.kend = w.p0 + a.T;
+    const kpos_t p0 = (kpos_t)w.p0, kend = (kpos_t)w.kend;
+    kpos_t lo = kend, hi = -1;
+    kpos_t lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
     for (int x = 0; x < 2; ++x) {
         if (!w.q[x].active) continue;
-        lo_x[x] = max(0, w.q[x].m0 - a.left);
-        hi_x[x] = min(a.T - 1, w.q[x].m0 + PP_BM - 1 + a.right);
+        lo_x[x] = max((kpos_t)0, (kpos_t)(p0 + w.q[x].m0 - a.left));
+        hi_x[x] = min(kend - 1, (kpos_t)(p0 + w.q[x].m0 + PP_BM - 1 + a.right));
         lo = min(lo, lo_x[x]);
         hi = max(hi, hi_x[x]);
     }
-    w.j_lo = lo / PP_BN;
-    w.n_tiles = hi / PP_BN - w.j_lo + 1;
+    w.j_lo = (int)(lo / PP_BN);
+    w.n_tiles = (int)(hi / PP_BN) - w.j_lo + 1;
     for (int x = 0; x < 2; ++x)
         if (w.q[x].active) {
-            w.q[x].ts = lo_x[x] / PP_BN - w.j_lo;
-            w.q[x].te = hi_x[x] / PP_BN - w.j_lo + 1;
+            w.q[x].ts = (int)(lo_x[x] / PP_BN) - w.j_lo;
+            w.q[x].te = (int)(hi_x[x] / PP_BN) - w.j_lo + 1;
         }
     w.hk = w.q[0].h / G;
     return w;
@@ -308,11 +339,16 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
     rescale = !first && atot != 1.f;
 }
 
-template <int D>
+// RING: a chunk of new tokens whose earlier keys are in the W-slot ring
+// (position p in slot p mod W): key tiles wholly in the chunk or wholly in
+// the ring (without wrapping round its end) come by TMA, the others by row
+// gathers.
+template <int D, bool RING>
 __global__ void __launch_bounds__(PP_THREADS, 1)
     swa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                          const TcPrefillArgs a)
+                          const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
+                          const TcPrefillArgs a, const RingArgs ring)
 {
     using C = PCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -324,7 +360,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const PPWork w = pp_make_work(a);
+    const PPWork w = pp_make_work<RING>(a, ring);
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -373,26 +409,64 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                                     w.q[x].m0, w.b);
                     }
         }
+        if (RING && lane == 0 && ring.pos[w.b] < 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+        // one K or V tile into stage st
+        auto load_tile = [&](bool is_v, int st, long long key0) {
+            uint8_t *dst = (is_v ? sV : sK) + st * C::KTILE;
+            uint64_t *bar = is_v ? &bars->v_full[st] : &bars->k_full[st];
+            if constexpr (RING) {
+                const bool ring_tile = key0 < w.p0;
+                const long long slot0 = ring_tile ? key0 % ring.W : 0;
+                if (!ring_tile || (key0 + PP_BN <= w.p0 && slot0 + PP_BN <= ring.W)) {
+                    SWA_DCHECK(ring_tile || key0 - w.p0 < a.T, a.ctl.status);
+                    if (lane == 0) {
+                        mbar_expect_tx(bar, C::KTILE);
+                        for (int ch = 0; ch < C::NCH; ++ch) {
+                            if (ring_tile)
+                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmVr : &tmKr, bar, ch * C::E, (int)slot0, w.hk,
+                                            w.b);
+                            else
+                                tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk,
+                                            (int)(key0 - w.p0), w.b);
+                        }
+                    }
+                    return;
+                }
+                // a tile that meets the chunk's first row or wraps round the
+                // ring's end: rows from wherever each position lives
+                const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(is_v ? a.v : a.k);
+                const __nv_bfloat16 *rc = static_cast<const __nv_bfloat16 *>(is_v ? ring.vc : ring.kc);
+                pp_gather_rows<D>(dst, src, lane, [&](int r) -> const __nv_bfloat16 * {
+                    const long long p = key0 + r;
+                    if (p >= w.p0) {
+                        const long long row = p - w.p0;
+                        return row < a.T ? src + (((long long)w.b * a.T + row) * a.Hkv + w.hk) * D : nullptr;
+                    }
+                    return rc + (((long long)w.b * a.Hkv + w.hk) * ring.W + p % ring.W) * D;
+                });
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar);
+            } else {
+                SWA_DCHECK(key0 >= 0 && key0 < a.T, a.ctl.status);
+                if (lane == 0) {
+                    mbar_expect_tx(bar, C::KTILE);
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk, (int)key0, w.b);
+                }
+            }
+        };
         for (int t = 0; t < w.n_tiles && ok; ++t) {
-            const int key0 = (w.j_lo + t) * PP_BN;
+            const long long key0 = (long long)(w.j_lo + t) * PP_BN;
             const int st = t % PP_NSTAGE;
             const uint32_t par = ((t / PP_NSTAGE) & 1) ^ 1;
             ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
             if (!ok) break;
-            SWA_DCHECK(key0 >= 0 && key0 < a.T, a.ctl.status);
-            if (lane == 0) {
-                mbar_expect_tx(&bars->k_full[st], C::KTILE);
-                for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_load_4d(sK + st * C::KTILE + ch * C::KCH, &tmK, &bars->k_full[st], ch * C::E, w.hk, key0, w.b);
-            }
+            load_tile(false, st, key0);
             kiss[st]++;
             ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
             if (!ok) break;
-            if (lane == 0) {
-                mbar_expect_tx(&bars->v_full[st], C::KTILE);
-                for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_load_4d(sV + st * C::KTILE + ch * C::KCH, &tmV, &bars->v_full[st], ch * C::E, w.hk, key0, w.b);
-            }
+            load_tile(true, st, key0);
             viss[st]++;
         }
         if (!ok && lane == 0) {
@@ -496,10 +570,15 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + pp_col_s(x);
         const uint32_t o_addr = tmem + lane_off + pp_col_o(x);
-        const int i_row = qt.m0 + r;            // query position
+        // key positions: 64-bit only for a chunk continuing a ring
+        typedef typename std::conditional<RING, long long, int>::type kpos_t;
+        const kpos_t p0 = RING ? (kpos_t)w.p0 : 0;
+        const kpos_t kend = RING ? (kpos_t)w.kend : (kpos_t)a.T;   // one past the last key
+        const int i_row = qt.m0 + r;            // row in q / o / lse
+        const kpos_t ip = p0 + i_row;           // query position
         const bool row_real = qt.active && r < qt.nrows;
         const bool warp_has_rows = qt.active && quarter * 32 < qt.nrows;
-        const int wi0 = qt.m0 + quarter * 32, wi1 = wi0 + 31;
+        const kpos_t wi0 = p0 + qt.m0 + quarter * 32, wi1 = wi0 + 31;
         float m = -CUDART_INF_F, l = 0.f;
         bool ok = true;
         int c = 0;
@@ -509,23 +588,23 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             // which 32-key chunks can any row of this warp see
-            const int key0 = (w.j_lo + t) * PP_BN;
+            const kpos_t key0 = (kpos_t)(w.j_lo + t) * PP_BN;
             int c_lo = 0, c_hi = -1;
             bool interior = false;
             if (warp_has_rows) {
-                const int lo = max(max(key0, wi0 - a.left), 0);
-                const int hi = min(min(key0 + PP_BN - 1, wi1 + a.right), a.T - 1);
+                const kpos_t lo = max(max(key0, (kpos_t)(wi0 - a.left)), (kpos_t)0);
+                const kpos_t hi = min(min(key0 + PP_BN - 1, (kpos_t)(wi1 + a.right)), kend - 1);
                 if (lo <= hi) {
-                    c_lo = (lo - key0) / 32;
-                    c_hi = (hi - key0) / 32;
+                    c_lo = (int)((lo - key0) / 32);
+                    c_hi = (int)((hi - key0) / 32);
                 }
-                interior = (key0 + PP_BN - 1 < a.T) && band_contains(wi1, key0, a.left, a.right) &&
+                interior = (key0 + PP_BN - 1 < kend) && band_contains(wi1, key0, a.left, a.right) &&
                            band_contains(wi0, key0 + PP_BN - 1, a.left, a.right);
             }
             SWA_DCHECK(c_lo >= 0 && c_hi < PP_BN / 32, a.ctl.status);
             // visible columns of this row
-            const int col_lo = max(i_row - a.left - key0, 0);
-            const int col_hi = min(min(i_row + a.right, a.T - 1) - key0, PP_BN - 1);
+            const int col_lo = (int)max(ip - a.left - key0, (kpos_t)0);
+            const int col_hi = (int)min(min((kpos_t)(ip + a.right), kend - 1) - key0, (kpos_t)(PP_BN - 1));
             bool rescale_o;
             float alpha;
             if (interior && c_lo == 0 && c_hi == PP_BN / 32 - 1)
@@ -608,18 +687,45 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
     }
 }
 
+// Ring cache [B,Hkv,W,D] bf16 viewed as (D, W, Hkv, B); box = one chunk of
+// 128 consecutive slots of one kv head.
 template <int D>
-cudaError_t launch_pp_d(const TcPrefillArgs &a, cudaStream_t s)
+bool pp_make_ring_map(CUtensorMap *m, const void *ptr, int B, int Hkv, int W)
 {
     using C = PCfg<D>;
-    CUtensorMap mq, mk, mv, mo;
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)Hkv, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)W * D * 2, (cuuint64_t)Hkv * W * D * 2};
+    cuuint32_t box[4] = {(cuuint32_t)C::E, (cuuint32_t)PP_BN, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     C::RB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, bool RING>
+cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
+{
+    using C = PCfg<D>;
+    CUtensorMap mq, mk, mv, mo, mkr, mvr;
     if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq, D, PP_BM) || !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv, D, PP_BN) ||
         !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv, D, PP_BN) || !make_bthd_map(&mo, a.o, a.B, a.T, a.Hq, D, PP_BM))
         return cudaErrorInvalidValue;
+    if (RING) {
+        if (!pp_make_ring_map<D>(&mkr, ring.kc, a.B, a.Hkv, ring.W) ||
+            !pp_make_ring_map<D>(&mvr, ring.vc, a.B, a.Hkv, ring.W))
+            return cudaErrorInvalidValue;
+    } else {
+        mkr = mk;   // unused without a ring
+        mvr = mv;
+    }
     static DeviceOnce once;
     cudaError_t e = once.get(
         [&](int) {
-            return cudaFuncSetAttribute(swa_prefill_pp_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            return cudaFuncSetAttribute(swa_prefill_pp_kernel<D, RING>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
         },
         nullptr);
@@ -629,7 +735,7 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, cudaStream_t s)
     const long long units = (long long)a.B * ((G % 2 == 0) ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    swa_prefill_pp_kernel<D><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a);
+    swa_prefill_pp_kernel<D, RING><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring);
     return cudaGetLastError();
 }
 
@@ -648,10 +754,16 @@ bool prefill_pp_applies(int d, const TcPrefillArgs &a)
     return (d == 32 || d == 64 || d == 128) && a.gidx == nullptr && a.g == 0 && a.left + a.right + 1 >= 256;
 }
 
-cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s)
+cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     if (!prefill_pp_applies(d, a)) return cudaErrorInvalidValue;
-    return d == 128 ? launch_pp_d<128>(a, s) : d == 64 ? launch_pp_d<64>(a, s) : launch_pp_d<32>(a, s);
+    if (ring.pos)
+        return d == 128 ? launch_pp_d<128, true>(a, ring, s)
+               : d == 64 ? launch_pp_d<64, true>(a, ring, s)
+                         : launch_pp_d<32, true>(a, ring, s);
+    return d == 128 ? launch_pp_d<128, false>(a, ring, s)
+           : d == 64 ? launch_pp_d<64, false>(a, ring, s)
+                     : launch_pp_d<32, false>(a, ring, s);
 }
 
 }  // namespace swa

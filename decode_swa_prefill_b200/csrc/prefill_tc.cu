@@ -1125,9 +1125,10 @@ cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArg
 cudaError_t launch_prefill_tc(int d, int mode, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     // a causal window of at most 64 keys: the single-pass kernel; windows of
-    // 256 keys or more without global keys: the 128-key kernel
+    // 256 keys or more without global keys (a chunk over a ring included):
+    // the 128-key kernel
     if (mode == 0 && ring.pos == nullptr && prefill_narrow_applies(d, a)) return launch_prefill_narrow(d, a, s);
-    if (mode == 0 && ring.pos == nullptr && prefill_pp_applies(d, a)) return launch_prefill_pp(d, a, s);
+    if (mode == 0 && prefill_pp_applies(d, a)) return launch_prefill_pp(d, a, ring, s);
 
     switch (d) {
     case 32: return launch_d<32>(mode, a, ring, s);

@@ -136,10 +136,11 @@ struct BwdArgs {
 cudaError_t launch_prefill_backward(int d, const BwdArgs &a, cudaStream_t s);
 
 // Band prefill with 128-key tiles and the two query tiles in alternation (no
-// global keys, sinks, ring or packed sequences): d = 32, 64 or 128 and
-// windows of at least 256 keys.
+// global keys, sinks or packed sequences; optionally a chunk continuing a
+// ring, ring.pos not null): d = 32, 64 or 128 and windows of at least 256
+// keys.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a);
-cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s);
 
 // Packed variable-length sequences (causal band mode): q/k/v/o are
 // [total,H,d] (TcPrefillArgs.T = total, B = number of sequences) and
