@@ -64,6 +64,10 @@ constexpr int PP_BN = 128;               // keys per key tile
 constexpr int PP_NSTAGE = 2;             // K and V pipeline depth
 constexpr int PP_THREADS = 320;
 constexpr float PP_RESCALE_LOG2 = 8.0f;  // raise the running max only beyond 2^8
+// where the keys come from: the prefill's own k/v; or (a chunk of new tokens)
+// its k/v and the W-slot ring before it; or its k/v plus one gathered tile
+// of the first n_sink positions (attention sinks)
+constexpr int PP_PLAIN = 0, PP_RING = 1, PP_SINKS = 2;
 
 template <int D>
 struct PCfg {
@@ -156,12 +160,21 @@ struct PPWork {
     int b, hk;
     PPTile q[2];
     int j_lo;      // first key tile (absolute, 128-key units)
+    int n_band;    // window key tiles; a sink tile follows them
     int n_tiles;   // key tiles the CTA streams
     long long p0;  // position of query row 0 (a chunk continuing a ring; else 0)
     long long kend; // one past the last key position (p0 + T)
 };
 
-__device__ __forceinline__ bool pp_active(const PPTile &q, int t) { return q.active && t >= q.ts && t < q.te; }
+// Does query tile q use key tile t (window tiles [ts, te), then the sink
+// tile, which every query tile takes)?
+template <int SRC>
+__device__ __forceinline__ bool pp_active(const PPTile &q, int n_band, int t)
+{
+    if constexpr (SRC == PP_SINKS)
+        if (t >= n_band) return q.active;
+    return q.active && t >= q.ts && t < q.te;
+}
 
 // Units: pairs of query heads of one kv head (even group size) or pairs of
 // consecutive row tiles of one head; query tiles in descending order, so the
@@ -169,9 +182,10 @@ __device__ __forceinline__ bool pp_active(const PPTile &q, int t) { return q.act
 // RING: the rows are a chunk of new tokens at positions pos[b] .. (a
 // negative entry is read as 0; the producer records it), and key tiles are
 // counted in absolute positions.
-template <bool RING>
+template <int SRC>
 __device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const RingArgs &ring)
 {
+    constexpr bool RING = SRC == PP_RING;
     PPWork w;
     const int G = a.Hq / a.Hkv;
     const int nqt = (a.T + PP_BM - 1) / PP_BM;
@@ -208,7 +222,8 @@ __device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const Rin
         hi = max(hi, hi_x[x]);
     }
     w.j_lo = (int)(lo / PP_BN);
-    w.n_tiles = (int)(hi / PP_BN) - w.j_lo + 1;
+    w.n_band = (int)(hi / PP_BN) - w.j_lo + 1;
+    w.n_tiles = w.n_band + ((SRC == PP_SINKS && a.g > 0) ? 1 : 0);
     for (int x = 0; x < 2; ++x)
         if (w.q[x].active) {
             w.q[x].ts = (int)(lo_x[x] / PP_BN) - w.j_lo;
@@ -343,7 +358,7 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_addr, int c_lo, int c
 // (position p in slot p mod W): key tiles wholly in the chunk or wholly in
 // the ring (without wrapping round its end) come by TMA, the others by row
 // gathers.
-template <int D, bool RING>
+template <int D, int SRC>
 __global__ void __launch_bounds__(PP_THREADS, 1)
     swa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -351,6 +366,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                           const TcPrefillArgs a, const RingArgs ring)
 {
     using C = PCfg<D>;
+    constexpr bool RING = SRC == PP_RING;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + C::OFF_Q;   // Q_X at sQ + X * QTILE
@@ -360,7 +376,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const PPWork w = pp_make_work<RING>(a, ring);
+    const PPWork w = pp_make_work<SRC>(a, ring);
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -456,17 +472,31 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 }
             }
         };
+        // the sink tile: positions 0 .. n_sink-1, zeros after
+        auto load_sinks = [&](bool is_v, int st) {
+            uint8_t *dst = (is_v ? sV : sK) + st * C::KTILE;
+            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(is_v ? a.v : a.k);
+            pp_gather_rows<D>(dst, src, lane, [&](int r) -> const __nv_bfloat16 * {
+                return r < a.g ? src + (((long long)w.b * a.T + r) * a.Hkv + w.hk) * D : nullptr;
+            });
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(is_v ? &bars->v_full[st] : &bars->k_full[st]);
+        };
         for (int t = 0; t < w.n_tiles && ok; ++t) {
             const long long key0 = (long long)(w.j_lo + t) * PP_BN;
             const int st = t % PP_NSTAGE;
             const uint32_t par = ((t / PP_NSTAGE) & 1) ^ 1;
+            const bool sink_tile = SRC == PP_SINKS && t >= w.n_band;
             ok = warp_wait_bounded(&bars->k_empty[st], par, ctl);
             if (!ok) break;
-            load_tile(false, st, key0);
+            if (sink_tile) load_sinks(false, st);
+            else load_tile(false, st, key0);
             kiss[st]++;
             ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
             if (!ok) break;
-            load_tile(true, st, key0);
+            if (sink_tile) load_sinks(true, st);
+            else load_tile(true, st, key0);
             viss[st]++;
         }
         if (!ok && lane == 0) {
@@ -526,7 +556,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             if (ok) {
                 tc_fence_after();
                 for (int x = 0; x < 2; ++x)
-                    if (pp_active(w.q[x], 0)) qk(x, 0);
+                    if (pp_active<SRC>(w.q[x], w.n_band, 0)) qk(x, 0);
                 if (leader) mma_commit(&bars->k_empty[0]);
             }
         }
@@ -539,18 +569,18 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             if (!ok) break;
             // tile A: PV of key tile t, then QK^T of key tile t+1 into the
             // same S columns (issue order keeps them apart)
-            if (pp_active(w.q[0], t)) ok = pv(0, t);
+            if (pp_active<SRC>(w.q[0], w.n_band, t)) ok = pv(0, t);
             if (!ok) break;
             if (more) {
                 tc_fence_after();
-                if (pp_active(w.q[0], t + 1)) qk(0, t + 1);
+                if (pp_active<SRC>(w.q[0], w.n_band, t + 1)) qk(0, t + 1);
             }
             // tile B likewise, half a step behind
-            if (pp_active(w.q[1], t)) ok = pv(1, t);
+            if (pp_active<SRC>(w.q[1], w.n_band, t)) ok = pv(1, t);
             if (!ok) break;
             if (leader) mma_commit(&bars->v_empty[st]);
             if (more) {
-                if (pp_active(w.q[1], t + 1)) qk(1, t + 1);
+                if (pp_active<SRC>(w.q[1], w.n_band, t + 1)) qk(1, t + 1);
                 if (leader) mma_commit(&bars->k_empty[(t + 1) % PP_NSTAGE]);
             }
             __syncwarp();
@@ -583,7 +613,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         bool ok = true;
         int c = 0;
         for (int t = 0; t < w.n_tiles && qt.active; ++t) {
-            if (!pp_active(qt, t)) continue;
+            if (!pp_active<SRC>(qt, w.n_band, t)) continue;
             ok = warp_wait_bounded(&bars->s_full[x], c & 1, ctl);
             if (!ok) break;
             tc_fence_after();
@@ -603,8 +633,18 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             }
             SWA_DCHECK(c_lo >= 0 && c_hi < PP_BN / 32, a.ctl.status);
             // visible columns of this row
-            const int col_lo = (int)max(ip - a.left - key0, (kpos_t)0);
-            const int col_hi = (int)min(min((kpos_t)(ip + a.right), kend - 1) - key0, (kpos_t)(PP_BN - 1));
+            int col_lo = (int)max(ip - a.left - key0, (kpos_t)0);
+            int col_hi = (int)min(min((kpos_t)(ip + a.right), kend - 1) - key0, (kpos_t)(PP_BN - 1));
+            if (SRC == PP_SINKS && t >= w.n_band) {
+                // sink positions 0 .. n_sink-1 below the row's window (the
+                // ones inside it were counted there; causal: all <= the row)
+                col_lo = 0;
+                col_hi = min(a.g, (int)(ip - a.left)) - 1;
+                const int last = warp_has_rows ? min(a.g, (int)(wi1 - a.left)) - 1 : -1;
+                c_lo = 0;
+                c_hi = last >= 0 ? last / 32 : -1;
+                interior = false;
+            }
             bool rescale_o;
             float alpha;
             if (interior && c_lo == 0 && c_hi == PP_BN / 32 - 1)
@@ -706,10 +746,11 @@ bool pp_make_ring_map(CUtensorMap *m, const void *ptr, int B, int Hkv, int W)
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool RING>
+template <int D, int SRC>
 cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     using C = PCfg<D>;
+    constexpr bool RING = SRC == PP_RING;
     CUtensorMap mq, mk, mv, mo, mkr, mvr;
     if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq, D, PP_BM) || !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv, D, PP_BN) ||
         !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv, D, PP_BN) || !make_bthd_map(&mo, a.o, a.B, a.T, a.Hq, D, PP_BM))
@@ -725,7 +766,7 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream
     static DeviceOnce once;
     cudaError_t e = once.get(
         [&](int) {
-            return cudaFuncSetAttribute(swa_prefill_pp_kernel<D, RING>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            return cudaFuncSetAttribute(swa_prefill_pp_kernel<D, SRC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
         },
         nullptr);
@@ -735,7 +776,7 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream
     const long long units = (long long)a.B * ((G % 2 == 0) ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    swa_prefill_pp_kernel<D, RING><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring);
+    swa_prefill_pp_kernel<D, SRC><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring);
     return cudaGetLastError();
 }
 
@@ -751,19 +792,28 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream
 // prefill (no global tokens) whose window spans at least 256 keys.
 bool prefill_pp_applies(int d, const TcPrefillArgs &a)
 {
-    return (d == 32 || d == 64 || d == 128) && a.gidx == nullptr && a.g == 0 && a.left + a.right + 1 >= 256;
+    // no global keys; attention sinks (gidx null, g > 0) with a causal window
+    // and at most one key tile of them
+    const bool keys_ok = a.gidx == nullptr && (a.g == 0 || (a.g <= PP_BN && a.right == 0));
+    return (d == 32 || d == 64 || d == 128) && keys_ok && a.left + a.right + 1 >= 256;
 }
 
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     if (!prefill_pp_applies(d, a)) return cudaErrorInvalidValue;
-    if (ring.pos)
-        return d == 128 ? launch_pp_d<128, true>(a, ring, s)
-               : d == 64 ? launch_pp_d<64, true>(a, ring, s)
-                         : launch_pp_d<32, true>(a, ring, s);
-    return d == 128 ? launch_pp_d<128, false>(a, ring, s)
-           : d == 64 ? launch_pp_d<64, false>(a, ring, s)
-                     : launch_pp_d<32, false>(a, ring, s);
+    if (ring.pos) {
+        if (a.g > 0) return cudaErrorInvalidValue;
+        return d == 128 ? launch_pp_d<128, PP_RING>(a, ring, s)
+               : d == 64 ? launch_pp_d<64, PP_RING>(a, ring, s)
+                         : launch_pp_d<32, PP_RING>(a, ring, s);
+    }
+    if (a.g > 0)
+        return d == 128 ? launch_pp_d<128, PP_SINKS>(a, ring, s)
+               : d == 64 ? launch_pp_d<64, PP_SINKS>(a, ring, s)
+                         : launch_pp_d<32, PP_SINKS>(a, ring, s);
+    return d == 128 ? launch_pp_d<128, PP_PLAIN>(a, ring, s)
+           : d == 64 ? launch_pp_d<64, PP_PLAIN>(a, ring, s)
+                     : launch_pp_d<32, PP_PLAIN>(a, ring, s);
 }
 
 }  // namespace swa

@@ -19,6 +19,11 @@ PREFILL_CASES = [
     (1, 130, 4, 1, 200, 3),    # window wider than T: sinks always inside it
     (1, 200, 2, 2, 1, 5),      # window of one token
     (1, 64, 4, 2, 16, 64),     # every token a sink: full causal attention
+    # windows of 256+ keys (the 128-key kernel with one gathered sink tile)
+    (1, 700, 8, 2, 256, 4),    # later rows see their sinks only through the sink tile
+    (2, 900, 4, 4, 300, 100),  # 100 sinks, inside the window for the first rows
+    (1, 400, 4, 1, 600, 8),    # window wider than T: the sink tile is all masked
+    (1, 1000, 8, 8, 257, 128), # a full sink tile
 ]
 
 
