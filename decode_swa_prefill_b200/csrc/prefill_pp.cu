@@ -67,7 +67,7 @@ constexpr float PP_RESCALE_LOG2 = 8.0f;  // raise the running max only beyond 2^
 // where the keys come from: the prefill's own k/v; or (a chunk of new tokens)
 // its k/v and the W-slot ring before it; or its k/v plus one gathered tile
 // of the first n_sink positions (attention sinks)
-constexpr int PP_PLAIN = 0, PP_RING = 1, PP_SINKS = 2;
+constexpr int PP_PLAIN = 0, PP_RING = 1, PP_SINKS = 2, PP_VARLEN = 3;
 
 template <int D>
 struct PCfg {
@@ -163,7 +163,7 @@ struct PPWork {
     int n_band;    // window key tiles; a sink tile follows them
     int n_tiles;   // key tiles the CTA streams
     long long p0;  // position of query row 0 (a chunk continuing a ring; else 0)
-    long long kend; // one past the last key position (p0 + T)
+    long long kend; // one past the last key position (p0 + T; a packed sequence: its length)
 };
 
 // Does query tile q use key tile t (window tiles [ts, te), then the sink
@@ -181,14 +181,17 @@ __device__ __forceinline__ bool pp_active(const PPTile &q, int n_band, int t)
 // short CTAs at the start of a causal sequence run last and fill the tail.
 // RING: the rows are a chunk of new tokens at positions pos[b] .. (a
 // negative entry is read as 0; the producer records it), and key tiles are
-// counted in absolute positions.
+// counted in absolute positions.  VARLEN: b is a packed sequence, tiles are
+// counted from its first row, and those past its end are inactive (an
+// inconsistent entry makes the sequence empty; the CTA records it).
 template <int SRC>
-__device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const RingArgs &ring)
+__device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl)
 {
     constexpr bool RING = SRC == PP_RING;
+    constexpr bool VARLEN = SRC == PP_VARLEN;
     PPWork w;
     const int G = a.Hq / a.Hkv;
-    const int nqt = (a.T + PP_BM - 1) / PP_BM;
+    const int nqt = ((VARLEN ? vl.max_len : a.T) + PP_BM - 1) / PP_BM;
     const int bid = blockIdx.x;
     for (int x = 0; x < 2; ++x) w.q[x] = PPTile{0, 0, 0, 0, 0, false};
     if (G % 2 == 0) {
@@ -206,17 +209,27 @@ __device__ __forceinline__ PPWork pp_make_work(const TcPrefillArgs &a, const Rin
             if (qt < nqt) w.q[x] = PPTile{h, qt * PP_BM, min(PP_BM, a.T - qt * PP_BM), 0, 0, true};
         }
     }
+    int left = a.left;
+    int TT = a.T;   // rows of this sequence
+    if constexpr (VARLEN) {
+        TT = varlen_ok(vl, w.b, a.T) ? vl.cu[w.b + 1] - vl.cu[w.b] : 0;
+        left = varlen_left(vl, w.b, a.left);
+        for (int x = 0; x < 2; ++x) {
+            if (w.q[x].m0 >= TT) w.q[x].active = false;
+            w.q[x].nrows = min(PP_BM, TT - w.q[x].m0);
+        }
+    }
     // positions: 64-bit only for a chunk continuing a ring
     typedef typename std::conditional<RING, long long, int>::type kpos_t;
     w.p0 = 0;
     if constexpr (RING) w.p0 = max((long long)ring.pos[w.b], 0LL);
-    w.kend = w.p0 + a.T;
+    w.kend = w.p0 + TT;
     const kpos_t p0 = (kpos_t)w.p0, kend = (kpos_t)w.kend;
     kpos_t lo = kend, hi = -1;
     kpos_t lo_x[2] = {0, 0}, hi_x[2] = {0, 0};
     for (int x = 0; x < 2; ++x) {
         if (!w.q[x].active) continue;
-        lo_x[x] = max((kpos_t)0, (kpos_t)(p0 + w.q[x].m0 - a.left));
+        lo_x[x] = max((kpos_t)0, (kpos_t)(p0 + w.q[x].m0 - left));
         hi_x[x] = min(kend - 1, (kpos_t)(p0 + w.q[x].m0 + PP_BM - 1 + a.right));
         lo = min(lo, lo_x[x]);
         hi = max(hi, hi_x[x]);
@@ -363,10 +376,11 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
     swa_prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                           const __grid_constant__ CUtensorMap tmKr, const __grid_constant__ CUtensorMap tmVr,
-                          const TcPrefillArgs a, const RingArgs ring)
+                          const TcPrefillArgs a, const RingArgs ring, const VarlenArgs vl)
 {
     using C = PCfg<D>;
     constexpr bool RING = SRC == PP_RING;
+    constexpr bool VARLEN = SRC == PP_VARLEN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + C::OFF_Q;   // Q_X at sQ + X * QTILE
@@ -376,7 +390,14 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const PPWork w = pp_make_work<SRC>(a, ring);
+    const PPWork w = pp_make_work<SRC>(a, ring, vl);
+    if constexpr (VARLEN) {
+        if (threadIdx.x == 0 && !varlen_ok(vl, w.b, a.T)) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
+        // a unit past its sequence's end has nothing to do
+        if (!w.q[0].active) return;
+    }
+    const int tb = VARLEN ? 0 : w.b;            // batch coordinate of the tensors
+    const int row0 = VARLEN ? vl.cu[w.b] : 0;   // tensor row of position 0
     WaitCtl ctl{&bars->abort, a.ctl.status, a.ctl.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -420,9 +441,9 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             for (int x = 0; x < 2; ++x)
                 if (w.q[x].active)
                     for (int ch = 0; ch < C::NCH; ++ch) {
-                        SWA_DCHECK(w.q[x].m0 >= 0 && w.q[x].m0 < a.T && w.q[x].h < a.Hq, a.ctl.status);
+                        SWA_DCHECK(w.q[x].m0 >= 0 && row0 + w.q[x].m0 < a.T && w.q[x].h < a.Hq, a.ctl.status);
                         tma_load_4d(sQ + x * C::QTILE + ch * C::QCH, &tmQ, &bars->q_full, ch * C::E, w.q[x].h,
-                                    w.q[x].m0, w.b);
+                                    row0 + w.q[x].m0, tb);
                     }
         }
         if (RING && lane == 0 && ring.pos[w.b] < 0) atomicMax(a.ctl.status, SWA_STATUS_BAD_INPUT);
@@ -464,11 +485,12 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar);
             } else {
-                SWA_DCHECK(key0 >= 0 && key0 < a.T, a.ctl.status);
+                SWA_DCHECK(key0 >= 0 && row0 + key0 < a.T, a.ctl.status);
                 if (lane == 0) {
                     mbar_expect_tx(bar, C::KTILE);
                     for (int ch = 0; ch < C::NCH; ++ch)
-                        tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk, (int)key0, w.b);
+                        tma_load_4d(dst + ch * C::KCH, is_v ? &tmV : &tmK, bar, ch * C::E, w.hk,
+                                    row0 + (int)key0, tb);
                 }
             }
         };
@@ -603,7 +625,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         // key positions: 64-bit only for a chunk continuing a ring
         typedef typename std::conditional<RING, long long, int>::type kpos_t;
         const kpos_t p0 = RING ? (kpos_t)w.p0 : 0;
-        const kpos_t kend = RING ? (kpos_t)w.kend : (kpos_t)a.T;   // one past the last key
+        const kpos_t kend = (RING || VARLEN) ? (kpos_t)w.kend : (kpos_t)a.T;   // one past the last key
+        const int left = VARLEN ? varlen_left(vl, w.b, a.left) : a.left;   // keys before the query
         const int i_row = qt.m0 + r;            // row in q / o / lse
         const kpos_t ip = p0 + i_row;           // query position
         const bool row_real = qt.active && r < qt.nrows;
@@ -622,18 +645,18 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             int c_lo = 0, c_hi = -1;
             bool interior = false;
             if (warp_has_rows) {
-                const kpos_t lo = max(max(key0, (kpos_t)(wi0 - a.left)), (kpos_t)0);
+                const kpos_t lo = max(max(key0, (kpos_t)(wi0 - left)), (kpos_t)0);
                 const kpos_t hi = min(min(key0 + PP_BN - 1, (kpos_t)(wi1 + a.right)), kend - 1);
                 if (lo <= hi) {
                     c_lo = (int)((lo - key0) / 32);
                     c_hi = (int)((hi - key0) / 32);
                 }
-                interior = (key0 + PP_BN - 1 < kend) && band_contains(wi1, key0, a.left, a.right) &&
-                           band_contains(wi0, key0 + PP_BN - 1, a.left, a.right);
+                interior = (key0 + PP_BN - 1 < kend) && band_contains(wi1, key0, left, a.right) &&
+                           band_contains(wi0, key0 + PP_BN - 1, left, a.right);
             }
             SWA_DCHECK(c_lo >= 0 && c_hi < PP_BN / 32, a.ctl.status);
             // visible columns of this row
-            int col_lo = (int)max(ip - a.left - key0, (kpos_t)0);
+            int col_lo = (int)max(ip - left - key0, (kpos_t)0);
             int col_hi = (int)min(min((kpos_t)(ip + a.right), kend - 1) - key0, (kpos_t)(PP_BN - 1));
             if (SRC == PP_SINKS && t >= w.n_band) {
                 // sink positions 0 .. n_sink-1 below the row's window (the
@@ -681,6 +704,9 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         // ---- epilogue: O / l -> bf16 -> shared memory -> TMA store ----
         if (ok && c > 0) ok = warp_wait_bounded(&bars->pv_done[x], (c - 1) & 1, ctl);
         uint8_t *stage = sQ + x * C::QTILE;    // Q_X is no longer read: its last QK^T is complete
+        // the last tile of a packed sequence is written row by row (a tile
+        // store would run into the next sequence)
+        const bool direct = VARLEN && qt.nrows < PP_BM;
         if (ok && qt.active) {
             tc_fence_after();
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -696,23 +722,32 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
                     pk.y = pack_bf16x2(ov[u * 8 + 2] * inv, ov[u * 8 + 3] * inv);
                     pk.z = pack_bf16x2(ov[u * 8 + 4] * inv, ov[u * 8 + 5] * inv);
                     pk.w = pack_bf16x2(ov[u * 8 + 6] * inv, ov[u * 8 + 7] * inv);
-                    *reinterpret_cast<uint4 *>(stage + pp_tile_offset<D>(r, cc * 16 + u * 8, C::QCH)) = pk;
+                    if (direct) {
+                        if (row_real) {
+                            SWA_DCHECK(row0 + i_row < a.T, a.ctl.status);
+                            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.o) +
+                                                 ((long long)(row0 + i_row) * a.Hq + qt.h) * D + cc * 16 + u * 8;
+                            *reinterpret_cast<uint4 *>(dst) = pk;
+                        }
+                    } else {
+                        *reinterpret_cast<uint4 *>(stage + pp_tile_offset<D>(r, cc * 16 + u * 8, C::QCH)) = pk;
+                    }
                 }
             }
             if (a.lse && row_real)
-                a.lse[((long long)w.b * a.Hq + qt.h) * a.T + i_row] =
+                a.lse[((long long)tb * a.Hq + qt.h) * a.T + row0 + i_row] =
                     (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
         // staging tile complete -> one thread per warpgroup stores it
         // (rows past T are clipped by the tensor map; an abort anywhere in
         // the CTA skips the store)
-        if (qt.active) {
+        if (!direct && qt.active) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->epi[x]);
             if (r == 0 && wait_bounded(&bars->epi[x], 0, ctl) && !bars->abort) {
                 for (int ch = 0; ch < C::NCH; ++ch)
-                    tma_store_4d(&tmO, stage + ch * C::QCH, ch * C::E, qt.h, qt.m0, w.b);
+                    tma_store_4d(&tmO, stage + ch * C::QCH, ch * C::E, qt.h, row0 + qt.m0, tb);
                 tma_store_commit();
                 tma_store_wait_all();
             }
@@ -747,13 +782,16 @@ bool pp_make_ring_map(CUtensorMap *m, const void *ptr, int B, int Hkv, int W)
 }
 
 template <int D, int SRC>
-cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
+cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl, cudaStream_t s)
 {
     using C = PCfg<D>;
     constexpr bool RING = SRC == PP_RING;
+    constexpr bool VARLEN = SRC == PP_VARLEN;
+    // packed sequences: the tensors as one sequence of `total` rows
+    const int TB = VARLEN ? 1 : a.B;
     CUtensorMap mq, mk, mv, mo, mkr, mvr;
-    if (!make_bthd_map(&mq, a.q, a.B, a.T, a.Hq, D, PP_BM) || !make_bthd_map(&mk, a.k, a.B, a.T, a.Hkv, D, PP_BN) ||
-        !make_bthd_map(&mv, a.v, a.B, a.T, a.Hkv, D, PP_BN) || !make_bthd_map(&mo, a.o, a.B, a.T, a.Hq, D, PP_BM))
+    if (!make_bthd_map(&mq, a.q, TB, a.T, a.Hq, D, PP_BM) || !make_bthd_map(&mk, a.k, TB, a.T, a.Hkv, D, PP_BN) ||
+        !make_bthd_map(&mv, a.v, TB, a.T, a.Hkv, D, PP_BN) || !make_bthd_map(&mo, a.o, TB, a.T, a.Hq, D, PP_BM))
         return cudaErrorInvalidValue;
     if (RING) {
         if (!pp_make_ring_map<D>(&mkr, ring.kc, a.B, a.Hkv, ring.W) ||
@@ -772,11 +810,15 @@ cudaError_t launch_pp_d(const TcPrefillArgs &a, const RingArgs &ring, cudaStream
         nullptr);
     if (e != cudaSuccess) return e;
     const int G = a.Hq / a.Hkv;
-    const int nqt = (a.T + PP_BM - 1) / PP_BM;
+    // units over (sequence, query tile [pair], head [pair]); for packed
+    // sequences the longest one sets the tiles and units past a sequence's
+    // end return at once
+    const int nqt = ((VARLEN ? vl.max_len : a.T) + PP_BM - 1) / PP_BM;
     const long long units = (long long)a.B * ((G % 2 == 0) ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
-    swa_prefill_pp_kernel<D, SRC><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring);
+    swa_prefill_pp_kernel<D, SRC><<<(int)units, PP_THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring,
+                                                                                  vl);
     return cudaGetLastError();
 }
 
@@ -801,19 +843,40 @@ bool prefill_pp_applies(int d, const TcPrefillArgs &a)
 cudaError_t launch_prefill_pp(int d, const TcPrefillArgs &a, const RingArgs &ring, cudaStream_t s)
 {
     if (!prefill_pp_applies(d, a)) return cudaErrorInvalidValue;
+    const VarlenArgs vl{nullptr, 0, nullptr};
     if (ring.pos) {
         if (a.g > 0) return cudaErrorInvalidValue;
-        return d == 128 ? launch_pp_d<128, PP_RING>(a, ring, s)
-               : d == 64 ? launch_pp_d<64, PP_RING>(a, ring, s)
-                         : launch_pp_d<32, PP_RING>(a, ring, s);
+        return d == 128 ? launch_pp_d<128, PP_RING>(a, ring, vl, s)
+               : d == 64 ? launch_pp_d<64, PP_RING>(a, ring, vl, s)
+                         : launch_pp_d<32, PP_RING>(a, ring, vl, s);
     }
     if (a.g > 0)
-        return d == 128 ? launch_pp_d<128, PP_SINKS>(a, ring, s)
-               : d == 64 ? launch_pp_d<64, PP_SINKS>(a, ring, s)
-                         : launch_pp_d<32, PP_SINKS>(a, ring, s);
-    return d == 128 ? launch_pp_d<128, PP_PLAIN>(a, ring, s)
-           : d == 64 ? launch_pp_d<64, PP_PLAIN>(a, ring, s)
-                     : launch_pp_d<32, PP_PLAIN>(a, ring, s);
+        return d == 128 ? launch_pp_d<128, PP_SINKS>(a, ring, vl, s)
+               : d == 64 ? launch_pp_d<64, PP_SINKS>(a, ring, vl, s)
+                         : launch_pp_d<32, PP_SINKS>(a, ring, vl, s);
+    return d == 128 ? launch_pp_d<128, PP_PLAIN>(a, ring, vl, s)
+           : d == 64 ? launch_pp_d<64, PP_PLAIN>(a, ring, vl, s)
+                     : launch_pp_d<32, PP_PLAIN>(a, ring, vl, s);
+}
+
+// Packed sequences (causal, no sinks): the call's window, clipped to the
+// longest sequence, or with one window per sequence the longest sequence
+// itself, spans at least 256 keys.  With one window per sequence the host
+// does not read the windows, so short ones run here too (correct, though
+// below 256 keys the 64-key kernel would be the faster one).
+bool prefill_pp_varlen_applies(int d, const TcPrefillArgs &a, const VarlenArgs &vl)
+{
+    return (d == 32 || d == 64 || d == 128) && vl.cu != nullptr && a.gidx == nullptr && a.g == 0 && a.right == 0 &&
+           a.left + 1 >= 256;
+}
+
+cudaError_t launch_prefill_pp_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s)
+{
+    if (!prefill_pp_varlen_applies(d, a, vl)) return cudaErrorInvalidValue;
+    const RingArgs ring{nullptr, nullptr, nullptr, 0};
+    return d == 128 ? launch_pp_d<128, PP_VARLEN>(a, ring, vl, s)
+           : d == 64 ? launch_pp_d<64, PP_VARLEN>(a, ring, vl, s)
+                     : launch_pp_d<32, PP_VARLEN>(a, ring, vl, s);
 }
 
 }  // namespace swa

@@ -172,22 +172,6 @@ __device__ __forceinline__ int tiles_of(const QTile &q, int n_glob)
     return q.active ? (q.te - q.ts) + n_glob : 0;
 }
 
-// Is packed sequence b's entry consistent (offsets inside the rows and
-// non-decreasing, length at most max_len, window at least 1)?
-__device__ __forceinline__ bool varlen_ok(const VarlenArgs &vl, int b, int total)
-{
-    const int c0 = vl.cu[b], c1 = vl.cu[b + 1];
-    return c0 >= 0 && c1 >= c0 && c1 <= total && c1 - c0 <= vl.max_len && (!vl.wseq || vl.wseq[b] >= 1);
-}
-
-// Keys before the query a row of packed sequence b sees: its own window's
-// (clipped to the longest sequence, like the call's single window), or the
-// call's.
-__device__ __forceinline__ int varlen_left(const VarlenArgs &vl, int b, int left)
-{
-    return vl.wseq ? min(max(vl.wseq[b], 1) - 1, vl.max_len) : left;
-}
-
 template <bool RING, bool SINKS, bool VARLEN>
 __device__ __forceinline__ Work make_work(const TcPrefillArgs &a, const RingArgs &ring, const VarlenArgs &vl,
                                           int n_mode1)
@@ -1111,6 +1095,7 @@ cudaError_t launch_d(int mode, const TcPrefillArgs &a, const RingArgs &ring, cud
 
 cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s)
 {
+    if (prefill_pp_varlen_applies(d, a, vl)) return launch_prefill_pp_varlen(d, a, vl, s);
     switch (d) {
     case 32: return launch_varlen_d<32>(a, vl, s);
     case 64: return launch_varlen_d<64>(a, vl, s);

@@ -152,6 +152,28 @@ struct VarlenArgs {
 };
 cudaError_t launch_prefill_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s);
 
+// Is packed sequence b's entry consistent (offsets inside the rows and
+// non-decreasing, length at most max_len, window at least 1)?
+__device__ __forceinline__ bool varlen_ok(const VarlenArgs &vl, int b, int total)
+{
+    const int c0 = vl.cu[b], c1 = vl.cu[b + 1];
+    return c0 >= 0 && c1 >= c0 && c1 <= total && c1 - c0 <= vl.max_len && (!vl.wseq || vl.wseq[b] >= 1);
+}
+
+// Keys before the query a row of packed sequence b sees: its own window's
+// (clipped to the longest sequence, like the call's single window), or the
+// call's.
+__device__ __forceinline__ int varlen_left(const VarlenArgs &vl, int b, int left)
+{
+    return vl.wseq ? min(max(vl.wseq[b], 1) - 1, vl.max_len) : left;
+}
+
+// The same calls on the 128-key kernel (prefill_pp.cu): d = 32, 64 or 128
+// and a call window (or, with one window per sequence, a longest sequence)
+// of at least 256 keys.
+bool prefill_pp_varlen_applies(int d, const TcPrefillArgs &a, const VarlenArgs &vl);
+cudaError_t launch_prefill_pp_varlen(int d, const TcPrefillArgs &a, const VarlenArgs &vl, cudaStream_t s);
+
 // ---- SIMT kernels ----
 // Attention sinks in the prefill calls: gidx == null with g > 0 means the
 // first g positions of each sequence are keys every later query sees

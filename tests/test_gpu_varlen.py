@@ -48,6 +48,35 @@ def test_varlen_f32(lengths):
     assert max_err(lse, ref_lse) <= 1e-5
 
 
+# windows of 256 keys or more run on the 128-key kernel: its tiles of a
+# sequence start at the sequence's first row, the last one is written row
+# by row, and units past a sequence's end do nothing
+WIDE = [
+    [700],
+    [1, 130, 0, 257, 640, 5],
+    [512, 512],
+    [17, 1000, 3, 300],
+]
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("lengths", WIDE)
+@pytest.mark.parametrize("W", [256, 300])
+def test_varlen_wide_window_bf16(d, lengths, W):
+    o, lse, ref_o, ref_lse = run(lengths, 8, 2, d, W, torch.bfloat16, seed=len(lengths) + d + W)
+    assert max_err(o, ref_o) <= tol_for(torch.bfloat16)
+    assert max_err(lse, ref_lse) <= 1e-2
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(3, 3), (4, 4), (8, 1)])
+def test_varlen_wide_window_group_sizes(Hq, Hkv):
+    # odd group size: a CTA holds two row tiles of one head, the second
+    # possibly past its sequence's end
+    o, lse, ref_o, ref_lse = run([129, 300, 77, 600], Hq, Hkv, 64, 256, torch.bfloat16, seed=Hq + 7 * Hkv)
+    assert max_err(o, ref_o) <= 2e-2
+    assert max_err(lse, ref_lse) <= 1e-2
+
+
 def test_odd_group_pairs_row_tiles():
     # group size 1: a CTA holds two row tiles of one head; the second may lie
     # past its sequence's end
@@ -65,11 +94,25 @@ def test_inconsistent_offsets_reported():
     assert swa.swa_get_device_status() == 0
 
 
+def test_inconsistent_offsets_reported_wide_window():
+    total, Hq, Hkv, d = 600, 2, 1, 64
+    q, k, v = (t[0].to(dev()) for t in wl.prefill_inputs(1, total, Hq, Hkv, d, torch.bfloat16, 8))
+    cu = torch.tensor([0, 300, 280, 600], dtype=torch.int32, device=dev())   # decreasing entry
+    assert swa.swa_get_device_status() == 0
+    swa.swa_prefill_varlen(q, k, v, cu, 256, 320)
+    assert swa.swa_get_device_status() == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_get_device_status() == 0
+
+
 # --------------------------------------------------- one window per sequence --
 
+# with one window per sequence the longest sequence picks the kernel: the
+# 128-key one from 256 rows (short windows there too), else the 64-key one
 MIXED = [
     ([1, 130, 0, 257, 64, 5], [1, 64, 7, 100, 200, 3]),   # window 1, one wider than its sequence, an empty sequence
     ([300, 300, 300], [33, 129, 300]),                    # windows below, across and at a 128-row tile
+    ([1, 130, 0, 200, 64, 5], [1, 64, 7, 100, 200, 3]),   # longest sequence below 256 rows
+    ([700, 129, 450], [256, 1000, 2]),                    # 128-key tiles, a 2-key window among them
 ]
 
 
@@ -124,19 +167,21 @@ def test_gemma_like_local_windows_in_one_batch():
     assert max_err(lse.cpu()[h, np.tile(r, Hq)], ref_lse) <= 2e-2
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_window_below_one_reported_and_rows_untouched(dtype):
-    lengths, windows = [100, 60, 90], [16, 0, 7]
+@pytest.mark.parametrize("dtype,lengths", [(torch.bfloat16, [100, 60, 90]), (torch.float32, [100, 60, 90]),
+                                           (torch.bfloat16, [300, 260, 290])])
+def test_window_below_one_reported_and_rows_untouched(dtype, lengths):
+    windows = [16, 0, 7] if lengths[0] < 256 else [300, 0, 17]
     total, Hq, Hkv, d = sum(lengths), 4, 2, 64
     q, k, v = (t[0].to(dev()) for t in wl.prefill_inputs(1, total, Hq, Hkv, d, dtype, 9))
-    cu = torch.tensor([0, 100, 160, 250], dtype=torch.int32, device=dev())
+    cu_list = [0] + np.cumsum(lengths).tolist()
+    cu = torch.tensor(cu_list, dtype=torch.int32, device=dev())
     win = torch.tensor(windows, dtype=torch.int32, device=dev())
     o = torch.full((total, Hq, d), 7.0, dtype=dtype, device=dev())
     assert swa.swa_get_device_status() == 0
-    swa.swa_prefill_varlen(q, k, v, cu, win, 100, o=o)
+    swa.swa_prefill_varlen(q, k, v, cu, win, max(lengths), o=o)
     assert swa.swa_get_device_status() == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_get_device_status() == 0
-    assert (o[100:160] == 7.0).all()                          # the sequence with window 0
-    ref, _ = oracle.swa_prefill_varlen(q.cpu(), k.cpu(), v.cpu(), [0, 100, 160, 250], [16, 1, 7])
-    keep = np.r_[0:100, 160:250]
+    assert (o[cu_list[1]:cu_list[2]] == 7.0).all()           # the sequence with window 0
+    ref, _ = oracle.swa_prefill_varlen(q.cpu(), k.cpu(), v.cpu(), cu_list, [windows[0], 1, windows[2]])
+    keep = np.r_[0:cu_list[1], cu_list[2]:total]
     assert max_err(o[keep], ref[keep]) <= tol_for(dtype)
