@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
 
     if (warp == 8) {
         // ------------------------------------------------------ producer --
-        int kiss[PP_NSTAGE] = {}, viss[PP_NSTAGE] = {};
+        int nk = 0, nv = 0;   // K and V tiles issued (tile t goes to stage t % PP_NSTAGE)
         bool ok = true;
         if (lane == 0) {
             int nq = 0;
@@ -514,18 +514,21 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
             if (!ok) break;
             if (sink_tile) load_sinks(false, st);
             else load_tile(false, st, key0);
-            kiss[st]++;
+            nk++;
             ok = warp_wait_bounded(&bars->v_empty[st], par, ctl);
             if (!ok) break;
             if (sink_tile) load_sinks(true, st);
             else load_tile(true, st, key0);
-            viss[st]++;
+            nv++;
         }
         if (!ok && lane == 0) {
             // let our own copies land before the CTA's shared memory goes away
             for (int s = 0; s < PP_NSTAGE; ++s) {
-                if (kiss[s] > 0) pp_drain_wait(&bars->k_full[s], (kiss[s] - 1) & 1, a.ctl.limit_ns);
-                if (viss[s] > 0) pp_drain_wait(&bars->v_full[s], (viss[s] - 1) & 1, a.ctl.limit_ns);
+                // copies issued into stage s: tiles s, s + PP_NSTAGE, ...
+                const int ks = nk > s ? (nk - s + PP_NSTAGE - 1) / PP_NSTAGE : 0;
+                const int vs = nv > s ? (nv - s + PP_NSTAGE - 1) / PP_NSTAGE : 0;
+                if (ks > 0) pp_drain_wait(&bars->k_full[s], (ks - 1) & 1, a.ctl.limit_ns);
+                if (vs > 0) pp_drain_wait(&bars->v_full[s], (vs - 1) & 1, a.ctl.limit_ns);
             }
         }
     } else if (warp == 9) {
