@@ -622,8 +622,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1)
         const int quarter = warp % 4;
         const int r = quarter * 32 + lane;      // row in tile = TMEM lane
         // a select, not w.q[x]: a run-time index would keep the work record
-        // in local memory (176 instead of 80 bytes of stack per thread, in
-        // an L1 that the 198 KB of shared memory leave small)
+        // in local memory (96 more bytes of stack per thread, in an L1 that
+        // the 198 KB of shared memory leave small)
         const PPTile qt = x ? w.q[1] : w.q[0];
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + pp_col_s(x);
