@@ -24,7 +24,7 @@ def run_causal(B, T, Hq, Hkv, d, W, dtype, seed, with_lse=True):
 
 @pytest.mark.parametrize("d", [32, 64, 128])
 @pytest.mark.parametrize("T,W", [(1, 1), (127, 5), (128, 128), (300, 40), (300, 1), (517, 200),
-                                 (400, 400), (257, 1000), (700, 256), (650, 255)])
+                                 (400, 400), (257, 1000), (700, 256), (650, 255), (1300, 1024), (1300, 1025)])
 def test_causal_bf16_small(d, T, W):
     o, lse, ref_o, ref_lse = run_causal(2, T, 4, 2, d, W, torch.bfloat16, seed=T * 7 + W + d)
     assert max_err(o, ref_o) <= 2e-2
@@ -115,7 +115,9 @@ def run_global(B, T, H, Hkv, d, W, g, dtype, seed, rows=None):
 @pytest.mark.parametrize("T,W,g", [(300, 64, 0), (300, 64, 5), (517, 100, 17), (130, 9, 1),
                                    (200, 2, 130), (64, 500, 3),
                                    # symmetric windows of 256+ keys without globals: the 128-key kernel
-                                   (300, 300, 0), (517, 600, 0), (260, 254, 0), (700, 256, 0)])
+                                   (300, 300, 0), (517, 600, 0), (260, 254, 0), (700, 256, 0),
+                                   # spans of 1023 and 1101 keys: either side of its persistent form
+                                   (1100, 1022, 0), (1400, 1100, 0)])
 def test_global_bf16_small(d, T, W, g):
     o, lse, ref_o, ref_lse = run_global(2, T, 3, 3, d, W, g, torch.bfloat16, seed=T + W + g + d)
     assert max_err(o, ref_o) <= 2e-2

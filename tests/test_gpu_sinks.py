@@ -24,6 +24,9 @@ PREFILL_CASES = [
     (2, 900, 4, 4, 300, 100),  # 100 sinks, inside the window for the first rows
     (1, 400, 4, 1, 600, 8),    # window wider than T: the sink tile is all masked
     (1, 1000, 8, 8, 257, 128), # a full sink tile
+    # windows of more than 1024 keys (the one-unit-per-CTA form of that kernel)
+    (1, 1400, 4, 2, 1100, 8),
+    (2, 1200, 4, 4, 1025, 100),
 ]
 
 

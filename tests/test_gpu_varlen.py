@@ -94,6 +94,16 @@ def test_inconsistent_offsets_reported():
     assert swa.swa_get_device_status() == 0
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("W", [1024, 1100])
+def test_varlen_long_window_bf16(d, W):
+    # a window of up to 1024 keys takes the persistent form of the 128-key
+    # kernel, a longer one the one-unit-per-CTA form
+    o, lse, ref_o, ref_lse = run([1300, 5, 1200, 129], 8, 2, d, W, torch.bfloat16, seed=d + W)
+    assert max_err(o, ref_o) <= tol_for(torch.bfloat16)
+    assert max_err(lse, ref_lse) <= 1e-2
+
+
 def test_inconsistent_offsets_reported_wide_window():
     total, Hq, Hkv, d = 600, 2, 1, 64
     q, k, v = (t[0].to(dev()) for t in wl.prefill_inputs(1, total, Hq, Hkv, d, torch.bfloat16, 8))
