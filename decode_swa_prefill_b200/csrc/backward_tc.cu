@@ -17,9 +17,11 @@
 // Three launches:
 //   bwd_delta_kernel   D_i = dout_i . o_i (fp32), one warp per row
 //   bwd_dq_kernel      one CTA per (batch, query head, 128-row query tile):
-//                      per 128-key tile S = Q K^T and dP = dO V^T into TMEM,
-//                      the elementwise warps turn them into dS (bf16, over
-//                      the S columns), then dQ += dS K accumulates in TMEM
+//                      per 128-key tile, in two halves of 64 keys, S = Q K^T
+//                      and dP = dO V^T into TMEM, the elementwise warps turn
+//                      them into dS (bf16, over the S columns), then dQ +=
+//                      dS K accumulates in TMEM; one half's elementwise pass
+//                      runs while the tensor core works on the other half
 //   bwd_dkdv_kernel    one CTA per (batch, kv head, 128-key tile): per
 //                      (query head of the group, 128-row query tile)
 //                      S^T = K Q^T and dP^T = V dO^T, then P^T and dS^T
@@ -61,8 +63,8 @@ struct BwdBars {
     uint64_t fixed_full;      // the CTA's own tiles (Q and dO, or K and V)
     uint64_t full[2];         // streamed tiles of a step
     uint64_t empty[2];
-    uint64_t s_full;          // S and dP (or their transposes) complete
-    uint64_t p_full;          // dS (and P) written (one arrival per warp)
+    uint64_t s_full[2];       // S and dP (or their transposes) complete [half of the key tile; dK/dV: [0]]
+    uint64_t p_full[2];       // dS (and P) written, one arrival per warp [likewise]
     uint64_t done;            // the last accumulating MMA complete
     uint32_t tmem_base;
     int abort;
@@ -101,6 +103,38 @@ __device__ __forceinline__ void bw_mma_acc(uint32_t d_tmem, uint32_t a_tmem, uin
 #pragma unroll
     for (int kk = 0; kk < BW_T / 16; ++kk)
         mma_bf16_ts(d_tmem, a_tmem + kk * 8, db_mn + (uint64_t)((kk * 16 * 128) >> 4), idesc,
+                    (acc_first || kk > 0) ? 1u : 0u);
+}
+
+// The same two products for one half of the key tile: d_tmem (64 columns) =
+// A B^T with B the 64 rows of the tile from row 64h (8-row swizzle atoms, so
+// the start moves by whole 1 KB blocks).
+template <int D>
+__device__ __forceinline__ void bw_mma_rows_half(uint32_t d_tmem, uint64_t da, uint64_t db, int h)
+{
+    using C = BCfg<D>;
+    constexpr uint32_t idesc = umma_idesc_bf16(BW_T, BW_T / 2, 0, 0);
+    const uint64_t dbh = db + (uint64_t)((h * (BW_T / 2) * 128) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const int byte = kk * 32;
+        const uint64_t off = (uint64_t)(((byte / 128) * C::CH + (byte % 128)) >> 4);
+        mma_bf16_ss(d_tmem, da + off, dbh + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// d_tmem += A B over the 64 contraction rows of half h: A (bf16, 128 rows x
+// 64) from TMEM at a_tmem, B rows 64h .. 64h+63 of a [128 rows][D] tile
+// read MN-major.
+template <int D>
+__device__ __forceinline__ void bw_mma_acc_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t db_mn, int h,
+                                                bool acc_first)
+{
+    constexpr uint32_t idesc = umma_idesc_bf16(BW_T, D, 0, 1);
+    const uint64_t dbh = db_mn + (uint64_t)((h * (BW_T / 2) * 128) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < BW_T / 32; ++kk)
+        mma_bf16_ts(d_tmem, a_tmem + kk * 8, dbh + (uint64_t)((kk * 16 * 128) >> 4), idesc,
                     (acc_first || kk > 0) ? 1u : 0u);
 }
 
@@ -160,8 +194,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 4);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bars->s_full[h], 1);
+            mbar_init(&bars->p_full[h], 4);
+        }
         mbar_init(&bars->done, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -213,26 +249,51 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const bool leader = lane == 0;
         const uint64_t dq = umma_smem_desc(smem_u32(sQ), 16, 8 * 128, UMMA_SW128);
         const uint64_t ddo = umma_smem_desc(smem_u32(sDO), 16, 8 * 128, UMMA_SW128);
-        bool ok = warp_wait_bounded(&bars->fixed_full, 0, ctl);
-        for (int t = 0; t < n && ok; ++t) {
-            const int st = t & 1;
-            ok = warp_wait_bounded(&bars->full[st], (t >> 1) & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
+        // Key tiles in two halves of 64 keys: S_h, dP_h into columns 64h and
+        // 128 + 64h, dS_h (bf16) over the first 32 of S_h's.  The next
+        // tile's half h is issued as soon as this tile's dQ += dS_h K_h is,
+        // so one half's elementwise pass runs while the tensor core works on
+        // the other half; the tensor core runs these MMAs in issue order, so
+        // no wait separates a dS read from the S write that follows it.
+        auto s_dp = [&](int st, int h) {
             const uint32_t ks = smem_u32(sKV + 2 * st * C::TILE), vs = ks + C::TILE;
+            bw_mma_rows_half<D>(tmem + 64 * h, dq, umma_smem_desc(ks, 16, 8 * 128, UMMA_SW128), h);        // S_h
+            bw_mma_rows_half<D>(tmem + 128 + 64 * h, ddo, umma_smem_desc(vs, 16, 8 * 128, UMMA_SW128), h); // dP_h
+            mma_commit(&bars->s_full[h]);
+        };
+        bool ok = warp_wait_bounded(&bars->fixed_full, 0, ctl);
+        if (ok && n > 0) ok = warp_wait_bounded(&bars->full[0], 0, ctl);
+        if (ok && n > 0) {
+            tc_fence_after();
             if (leader) {
-                bw_mma_rows<D>(tmem, dq, umma_smem_desc(ks, 16, 8 * 128, UMMA_SW128));         // S  = Q K^T
-                bw_mma_rows<D>(tmem + 128, ddo, umma_smem_desc(vs, 16, 8 * 128, UMMA_SW128));  // dP = dO V^T
-                mma_commit(&bars->s_full);
+                s_dp(0, 0);
+                s_dp(0, 1);
             }
             __syncwarp();
-            ok = warp_wait_bounded(&bars->p_full, t & 1, ctl);
+        }
+        for (int t = 0; t < n && ok; ++t) {
+            const int st = t & 1;
+            const bool more = t + 1 < n;
+            const uint32_t ks = smem_u32(sKV + 2 * st * C::TILE);
+            const uint64_t dk_mn = umma_smem_desc(ks, C::CH, 8 * 128, UMMA_SW128);
+            // half 0: dQ += dS_0 K_0, then the next tile's S_0, dP_0
+            ok = warp_wait_bounded(&bars->p_full[0], t & 1, ctl);
+            if (ok && more) ok = warp_wait_bounded(&bars->full[st ^ 1], ((t + 1) >> 1) & 1, ctl);
             if (!ok) break;
             tc_fence_after();
             if (leader) {
-                // dQ += dS K (dS: bf16 over the first 64 S columns)
-                bw_mma_acc<D>(tmem + 256, tmem, umma_smem_desc(ks, C::CH, 8 * 128, UMMA_SW128), t > 0);
+                bw_mma_acc_half<D>(tmem + 256, tmem, dk_mn, 0, t > 0);
+                if (more) s_dp(st ^ 1, 0);
+            }
+            __syncwarp();
+            // half 1: dQ += dS_1 K_1; the stage is free; the next tile's S_1, dP_1
+            ok = warp_wait_bounded(&bars->p_full[1], t & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            if (leader) {
+                bw_mma_acc_half<D>(tmem + 256, tmem + 64, dk_mn, 1, true);
                 mma_commit(&bars->empty[st]);
+                if (more) s_dp(st ^ 1, 1);
             }
             __syncwarp();
         }
@@ -250,33 +311,39 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const float lse2 = i < a.T ? a.lse[rowid] * 1.4426950408889634f : CUDART_INF_F;
         const float dl = i < a.T ? a.delta[rowid] : 0.f;
         bool ok = true;
-        for (int t = 0; t < n; ++t) {
-            ok = warp_wait_bounded(&bars->s_full, t & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
+        for (int t = 0; t < n && ok; ++t) {
             const int key0 = (t0 + t) * BW_T;
+            for (int h = 0; h < 2; ++h) {
+                ok = warp_wait_bounded(&bars->s_full[h], t & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
-                float s[32], dp[32];
-                tmem_ld32(tmem + lane_off + cc * 32, s);
-                tmem_ld32(tmem + lane_off + 128 + cc * 32, dp);
-                tmem_ld_wait_dep(s);
-                reg_fence32(dp);
-                uint32_t pk[16];
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int cc = 2 * h + c2;   // 32-key chunk of the tile
+                    float s[32], dp[32];
+                    tmem_ld32(tmem + lane_off + cc * 32, s);
+                    tmem_ld32(tmem + lane_off + 128 + cc * 32, dp);
+                    tmem_ld_wait_dep(s);
+                    reg_fence32(dp);
+                    uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int j = key0 + cc * 32 + e;
-                    const float p0 = bw_allowed(i, j, a.T, a.left, a.right) ? ex2_approx(s[e] * a.scale_log2 - lse2) : 0.f;
-                    const float p1 =
-                        bw_allowed(i, j + 1, a.T, a.left, a.right) ? ex2_approx(s[e + 1] * a.scale_log2 - lse2) : 0.f;
-                    pk[e / 2] = pack_bf16x2(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
+                    for (int e = 0; e < 32; e += 2) {
+                        const int j = key0 + cc * 32 + e;
+                        const float p0 =
+                            bw_allowed(i, j, a.T, a.left, a.right) ? ex2_approx(s[e] * a.scale_log2 - lse2) : 0.f;
+                        const float p1 = bw_allowed(i, j + 1, a.T, a.left, a.right)
+                                             ? ex2_approx(s[e + 1] * a.scale_log2 - lse2)
+                                             : 0.f;
+                        pk[e / 2] = pack_bf16x2(p0 * (dp[e] - dl), p1 * (dp[e + 1] - dl));
+                    }
+                    // dS of this half: bf16 pairs from column 64h on
+                    tmem_st16u(tmem + lane_off + 64 * h + c2 * 16, pk);
                 }
-                tmem_st16u(tmem + lane_off + cc * 16, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full[h]);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full);
         }
         // ---- epilogue: dQ * scale -> bf16 ----
         // (the TMEM loads are warp-wide: every lane takes part, rows past T
@@ -350,8 +417,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 4);
+        mbar_init(&bars->s_full[0], 1);
+        mbar_init(&bars->p_full[0], 4);
         mbar_init(&bars->done, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -423,10 +490,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             if (leader) {
                 bw_mma_rows<D>(tmem, dk, umma_smem_desc(qs, 16, 8 * 128, UMMA_SW128));        // S^T  = K Q^T
                 bw_mma_rows<D>(tmem + 128, dv, umma_smem_desc(gs, 16, 8 * 128, UMMA_SW128));  // dP^T = V dO^T
-                mma_commit(&bars->s_full);
+                mma_commit(&bars->s_full[0]);
             }
             __syncwarp();
-            ok = warp_wait_bounded(&bars->p_full, s & 1, ctl);
+            ok = warp_wait_bounded(&bars->p_full[0], s & 1, ctl);
             if (!ok) break;
             tc_fence_after();
             if (leader) {
@@ -449,7 +516,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         bool ok = true;
         for (int s = 0; s < nsteps; ++s) {
-            ok = warp_wait_bounded(&bars->s_full, s & 1, ctl);
+            ok = warp_wait_bounded(&bars->s_full[0], s & 1, ctl);
             if (!ok) break;
             tc_fence_after();
             const int m0 = (u0 + s % nu) * BW_T;
@@ -480,7 +547,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->p_full);
+            if (lane == 0) mbar_arrive(&bars->p_full[0]);
         }
         // ---- epilogue: dK * scale, dV -> bf16 ----
         // (the TMEM loads are warp-wide: every lane takes part, keys past T
