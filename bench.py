@@ -874,6 +874,7 @@ PROFILE_CASES = {
     # few GB at most so that an ncu capture of one launch ends quickly
     "prefill_small": (wl.MISTRAL_PREFILL, {"T": 8192}),
     "prefill": (wl.MISTRAL_PREFILL, {}),
+    "prefill_w512": (wl.MISTRAL_PREFILL, {"T": 16384, "W": 512}),   # the persistent form
     "longformer": (wl.LONGFORMER, {}),
     "tinymistral": (wl.TINYMISTRAL, {}),
     "chunk": (wl.MISTRAL_CHUNK, {}),
