@@ -15,7 +15,7 @@
 // O(T W d) like the forward pass.
 //
 // Three launches:
-//   bwd_delta_kernel   D_i = dout_i . o_i (fp32), one warp per row
+//   bwd_delta_kernel   D_i = dout_i . o_i (fp32), 16-byte loads, D/8 lanes per row
 //   bwd_dq_kernel      one CTA per (batch, query head, 128-row query tile):
 //                      per 128-key tile, in two halves of 64 keys, S = Q K^T
 //                      and dP = dO V^T into TMEM, the elementwise warps turn
@@ -144,24 +144,47 @@ __device__ __forceinline__ bool bw_allowed(int i, int j, int T, int left, int ri
 }
 
 // ------------------------------------------------------------ D_i = dO.O --
+// D/8 lanes per row, 16 bytes each; a warp takes BW_DPASS groups of 32/(D/8)
+// consecutive rows, all loads issued before the first product.
+constexpr int BW_DPASS = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *dout, const __nv_bfloat16 *o,
                                                          float *delta, int B, int T, int Hq)
 {
-    const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;   // (b*T + i)*Hq + h
+    constexpr int LPR = D / 8;        // lanes per row
+    constexpr int RPW = 32 / LPR;     // rows per warp and pass
+    const long long rows = (long long)B * T * Hq;   // row = (b*T + i)*Hq + h
     const int lane = threadIdx.x % 32;
-    if (row >= (long long)B * T * Hq) return;
-    constexpr int EPL = D / 32;
-    const __nv_bfloat16 *g = dout + row * D + lane * EPL;
-    const __nv_bfloat16 *x = o + row * D + lane * EPL;
-    float acc = 0.f;
+    const long long r0 = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * RPW * BW_DPASS + lane / LPR;
+    const int e0 = (lane % LPR) * 8;
+    uint4 g[BW_DPASS], x[BW_DPASS];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc += __bfloat162float(g[e]) * __bfloat162float(x[e]);
+    for (int p = 0; p < BW_DPASS; ++p) {
+        const long long row = r0 + (long long)p * RPW;
+        g[p] = make_uint4(0, 0, 0, 0);
+        x[p] = make_uint4(0, 0, 0, 0);
+        if (row < rows) {
+            g[p] = __ldg(reinterpret_cast<const uint4 *>(dout + row * D + e0));
+            x[p] = __ldg(reinterpret_cast<const uint4 *>(o + row * D + e0));
+        }
+    }
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (lane == 0) {
-        const long long h = row % Hq, bi = row / Hq, i = bi % T, b = bi / T;
-        delta[(b * Hq + h) * T + i] = acc;
+    for (int p = 0; p < BW_DPASS; ++p) {
+        const uint32_t gu[4] = {g[p].x, g[p].y, g[p].z, g[p].w}, xu[4] = {x[p].x, x[p].y, x[p].z, x[p].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            acc += __uint_as_float(gu[k] << 16) * __uint_as_float(xu[k] << 16);
+            acc += __uint_as_float(gu[k] & 0xffff0000u) * __uint_as_float(xu[k] & 0xffff0000u);
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const long long row = r0 + (long long)p * RPW;
+        if (lane % LPR == 0 && row < rows) {
+            const long long h = row % Hq, bi = row / Hq, i = bi % T, b = bi / T;
+            delta[(b * Hq + h) * T + i] = acc;
+        }
     }
 }
 
@@ -627,7 +650,9 @@ cudaError_t launch_bwd_d(const BwdArgs &a, cudaStream_t s)
         nullptr);
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.T * a.Hq;
-    bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.dout),
+    const long long rows_per_block = 8LL * (32 / (D / 8)) * BW_DPASS;
+    bwd_delta_kernel<D><<<(unsigned)((rows + rows_per_block - 1) / rows_per_block), 256, 0, s>>>(
+                                                                   static_cast<const __nv_bfloat16 *>(a.dout),
                                                                    static_cast<const __nv_bfloat16 *>(a.o), a.delta,
                                                                    a.B, a.T, a.Hq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
