@@ -9,7 +9,7 @@
 // page and of the Ultralytics glossary's FlashAttention entry).  Work per
 // query tile is O(W*d), total O(T*W*d).
 //
-// CTA anatomy (352 threads, one CTA per SM), two 128-row query tiles X = A, B
+// CTA anatomy (384 threads, one CTA per SM), two 128-row query tiles X = A, B
 // that share one kv head, hence every K/V tile: the two query heads of a GQA
 // pair at the same rows, or (odd group size) two consecutive row tiles of one
 // head, whose key ranges are then merged.
@@ -20,6 +20,10 @@
 //   warp 9     TMEM allocator; with warp 10, the MMA issuers: warp 9 + X runs
 //              tile X's schedule and its lane 0 issues X's tcgen05.mma, so a
 //              wait on one tile never holds up the other tile's MMAs
+//   warp 11    idle: it completes warpgroup 2 (warps 8-11), which hands
+//              registers to the softmax warpgroups (setmaxnreg) -- three
+//              warps on a sub-partition cap a thread at 168 registers, where
+//              the softmax spilled
 // TMEM (all 512 columns):
 //   S[X][b]  columns 128X + 64b: fp32 scores of one 64-key tile, b = buffer
 //   P[X][b]  the first 32 columns of S[X][b]: bf16 probabilities (pairs)
@@ -64,7 +68,13 @@ namespace {
 constexpr int BM = 128;              // query rows per tile (= TMEM lanes)
 constexpr int BN = 64;               // keys per key tile
 constexpr int NSTAGE = 3;            // K and V pipeline depth
-constexpr int NTHREADS = 352;
+constexpr int NTHREADS = 384;
+// registers per thread after the split: 256 x 200 + 128 x 104 = 384 x 168,
+// the block's launch total (checked on the host before each launch: an
+// increase the block cannot cover would wait for ever).  Measured against
+// 11 warps at 168: Longformer prefill 0.316 -> 0.293 ms, causal W = 128 (d
+// = 128) 0.201 -> 0.193 ms, W = 192 (d = 64) 0.190 -> 0.180 ms (T = 16384).
+constexpr int TC_REG_SOFTMAX = 200, TC_REG_OTHER = 104;
 constexpr float RESCALE_LOG2 = 8.0f; // raise the running max only beyond 2^8
 constexpr int POLY_EVERY = 4;        // every 4th pair of exponentials on the FMA pipe
 constexpr int SM_SMEM = 228 * 1024;  // shared memory per SM
@@ -520,6 +530,8 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
 
     const int32_t *gb = a.gidx ? a.gidx + (long long)w.b * a.g : nullptr;
 
+    // warpgroup 2 (producer, MMA issuers, idle warp 11) gives registers up
+    if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(TC_REG_OTHER) : "memory");
     if (warp == 8) {
         // ------------------------------------------------------ producer --
         int kiss[NSTAGE] = {}, viss[NSTAGE] = {};
@@ -753,7 +765,9 @@ __device__ __forceinline__ void prefill_cta(const CUtensorMap *tmQ, const CUtens
             drain_wait(&bars->drain[x], 0, a.ctl.limit_ns);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
+        // the softmax warpgroups take them
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(TC_REG_SOFTMAX) : "memory");
         // ------------------------------------------- softmax + epilogue --
         const int x = warp / 4;                 // query tile of this warpgroup
         const int quarter = warp % 4;
@@ -1047,6 +1061,14 @@ cudaError_t launch_dr(int mode, const TcPrefillArgs &a, const RingArgs &ring, cu
     }
     const int grid = n_mode0 + n_mode1;
     if (grid == 0) return cudaSuccess;
+    {
+        const void *kfn = RING ? (const void *)swa_prefill_ring_kernel<D>
+                          : sinks ? (const void *)swa_prefill_sinks_kernel<D> : (const void *)swa_prefill_tc_kernel<D>;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kfn) != cudaSuccess ||
+            fa.numRegs * NTHREADS < 256 * TC_REG_SOFTMAX + 128 * TC_REG_OTHER)
+            return cudaErrorInvalidConfiguration;
+    }
     if (RING)
         swa_prefill_ring_kernel<D><<<grid, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, mkr, mvr, a, ring, n_mode1);
     else if (sinks)
@@ -1081,6 +1103,12 @@ cudaError_t launch_varlen_d(const TcPrefillArgs &a, const VarlenArgs &vl, cudaSt
     const long long units = (long long)a.B * (pair_heads ? (a.Hq / 2) * nqt : a.Hq * ((nqt + 1) / 2));
     if (units == 0) return cudaSuccess;
     if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, (const void *)swa_prefill_varlen_kernel<D>) != cudaSuccess ||
+            fa.numRegs * NTHREADS < 256 * TC_REG_SOFTMAX + 128 * TC_REG_OTHER)
+            return cudaErrorInvalidConfiguration;
+    }
     swa_prefill_varlen_kernel<D><<<(int)units, NTHREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, mo, a, vl, 0);
     return cudaGetLastError();
 }
